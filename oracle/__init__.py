@@ -1,0 +1,240 @@
+"""Oracle: slow, plain fp64 CPU reference for Parallax attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline legs of ``bench.py`` may import this package.  The product path
+(``covariance_corrected_softmax_b200``) never imports it and shares no code with
+it; the only thing both sides share is the seeded input generator module, which
+holds none of the method's arithmetic.
+
+The arithmetic lives in ``plx_oracle.c`` (fp64, one query row at a time).  This
+module only marshals layouts into the C routine's "key stream" form and applies
+the two layout readings the pages leave open:
+
+* GQA head mapping: query head ``h`` reads key/value head ``h // (H_q // H_kv)``
+  (consecutive query heads share a KV head).  The pages never mention grouped
+  heads; this is the plainest reading of a multi-head operator with fewer KV
+  heads than query heads.
+* Key sets: causal prefill row ``i`` sees keys ``0..i``; non-causal sees all
+  ``L``; decode of batch ``b`` sees cache rows ``0..seqlen_b-1`` with ``seqlen_b``
+  clamped to ``[0, S_max]``; an empty set gives ``out = 0`` and ``lse = -inf``.
+
+Operator (page 1 "Parallax: Parameterized Local Linear Attention Gives
+Transformers a 'Second Eye'", section 1.3; page 3 "Parallax keeps softmax, adds
+covariance correction branch"): ``out_i = o_SA,i - Sigma_KV^(i)^T rho_i`` with
+``Sigma_KV^(i) = sum_j a_ij (k_j - mu_i)(v_j - o_SA,i)^T``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "plx_oracle.c")
+_LIB = os.path.join(_HERE, "libplx_oracle.so")
+
+FORM_EXPLICIT = 0  # forms the d_k x d_v covariance matrix (the definition)
+FORM_EXPANDED = 1  # o - (sum a t v - (sum a t) o): the one-pass rewrite
+_FORMS = {"explicit": FORM_EXPLICIT, "expanded": FORM_EXPANDED}
+
+
+def build(src: str = _SRC, out: str = _LIB, extra_flags: Sequence[str] = ()) -> str:
+    """Compile the C oracle with gcc into a shared library; returns its path."""
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", *extra_flags,
+           "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+class Oracle:
+    """Handle on one compiled copy of the C oracle (tests may load mutants)."""
+
+    def __init__(self, lib_path: str = _LIB):
+        if lib_path == _LIB and (not os.path.exists(_LIB)
+                                 or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)):
+            build()
+        self.path = lib_path
+        self._lib = ctypes.CDLL(lib_path)
+        f = self._lib.plxo_rows
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int64)
+        f.argtypes = [dp, dp, dp, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                      ctypes.c_int, ip, ip, ctypes.c_int64, ctypes.c_double,
+                      ctypes.c_int, dp, dp, ctypes.c_int]
+        f.restype = ctypes.c_int
+        self._rows = f
+
+    # ------------------------------------------------------------------ core
+    def rows(self, q, rho, k, v, row_stream, row_nkeys, scale: float,
+             form: str = "explicit", threads: Optional[int] = None
+             ) -> Tuple[np.ndarray, np.ndarray]:
+        """Evaluate query rows against key/value streams.
+
+        q, rho: [R, dk]; k: [P, S, dk]; v: [P, S, dv]; row_stream, row_nkeys: [R].
+        Returns (out [R, dv], lse [R]) in float64.
+        """
+        q = _f64(q)
+        rho = _f64(rho)
+        k = _f64(k)
+        v = _f64(v)
+        R, dk = q.shape
+        P, S, dk2 = k.shape
+        dv = v.shape[2]
+        assert rho.shape == (R, dk) and dk2 == dk and v.shape[:2] == (P, S)
+        rs = np.ascontiguousarray(np.asarray(row_stream, dtype=np.int64).reshape(R))
+        rn = np.ascontiguousarray(np.asarray(row_nkeys, dtype=np.int64).reshape(R))
+        out = np.zeros((R, dv), dtype=np.float64)
+        lse = np.zeros((R,), dtype=np.float64)
+        if R == 0:
+            return out, lse
+        if P == 0:  # no streams: every row must be empty
+            assert np.all(rn == 0)
+            k = np.zeros((1, max(S, 1), dk))
+            v = np.zeros((1, max(S, 1), dv))
+            P, S = 1, max(S, 1)
+            rs = np.zeros_like(rs)
+        rc = self._rows(_p(q), _p(rho), _p(k), _p(v), P, S, dk, dv,
+                        rs.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                        rn.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
+                        float(scale), _FORMS[form], _p(out), _p(lse),
+                        int(threads or default_threads()))
+        if rc != 0:
+            raise ValueError("oracle rejected its arguments")
+        return out, lse
+
+    # --------------------------------------------------------------- layouts
+    def prefill(self, q, rho, k, v, causal: bool, scale: float, rows=None,
+                form: str = "explicit", threads: Optional[int] = None):
+        """Prefill rows.  q, rho: [B, L, Hq, dk]; k: [B, L, Hkv, dk]; v: [B, L, Hkv, dv].
+
+        rows: None (all rows; returns out [B, L, Hq, dv], lse [B, Hq, L]) or an
+        int array [R, 3] of (b, h, i) (returns out [R, dv], lse [R]).
+        """
+        B, L, Hq, dk = q.shape
+        Hkv = k.shape[2]
+        assert Hq % Hkv == 0, "H_q must be a multiple of H_kv"
+        G = Hq // Hkv
+        full = rows is None
+        if full:
+            bb, ii, hh = np.meshgrid(np.arange(B), np.arange(L), np.arange(Hq), indexing="ij")
+            rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1)
+        rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+        b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+        hk = h // G
+        nkeys = (i + 1) if causal else np.full_like(i, L)
+        sid, ks, vs = _streams(k, v, b, hk, int(nkeys.max()) if len(nkeys) else 0)
+        out, lse = self.rows(_take(q, (b, i, h)), _take(rho, (b, i, h)), ks, vs, sid, nkeys,
+                             scale, form, threads)
+        if full:
+            out = out.reshape(B, L, Hq, -1)
+            lse = lse.reshape(B, L, Hq).transpose(0, 2, 1).copy()
+        return out, lse
+
+    def decode(self, q, rho, k_cache, v_cache, seqlens, scale: float, rows=None,
+               form: str = "explicit", threads: Optional[int] = None):
+        """Single-token decode.  q, rho: [B, Hq, dk]; caches: [B, S_max, Hkv, d].
+
+        rows: None (all; returns out [B, Hq, dv], lse [B, Hq]) or an int array
+        [R, 2] of (b, h) (returns out [R, dv], lse [R]).
+        """
+        B, Hq, dk = q.shape
+        S_max, Hkv = k_cache.shape[1], k_cache.shape[2]
+        assert Hq % Hkv == 0, "H_q must be a multiple of H_kv"
+        G = Hq // Hkv
+        sl = np.clip(np.asarray(_np(seqlens)).astype(np.int64).reshape(B), 0, S_max)
+        full = rows is None
+        if full:
+            bb, hh = np.meshgrid(np.arange(B), np.arange(Hq), indexing="ij")
+            rows = np.stack([bb.ravel(), hh.ravel()], axis=1)
+        rows = np.asarray(rows, dtype=np.int64).reshape(-1, 2)
+        b, h = rows[:, 0], rows[:, 1]
+        nkeys = sl[b]
+        sid, ks, vs = _streams(k_cache, v_cache, b, h // G, int(nkeys.max()) if len(nkeys) else 0)
+        out, lse = self.rows(_take(q, (b, h)), _take(rho, (b, h)), ks, vs, sid, nkeys,
+                             scale, form, threads)
+        if full:
+            out = out.reshape(B, Hq, -1)
+            lse = lse.reshape(B, Hq)
+        return out, lse
+
+
+def _np(x):
+    """numpy view of a numpy array or a (CPU or device) torch tensor, exact values."""
+    if isinstance(x, np.ndarray):
+        return x
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu")
+            if x.dtype in (torch.bfloat16, torch.float16):
+                x = x.to(torch.float32)  # exact
+            return x.numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x)
+
+
+def _f64(x) -> np.ndarray:
+    return np.ascontiguousarray(_np(x), dtype=np.float64)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _take(x, idx):
+    """x[idx] for integer index arrays, gathered before any host copy."""
+    if isinstance(x, np.ndarray):
+        return x[idx]
+    import torch
+    tidx = tuple(torch.as_tensor(np.asarray(a), dtype=torch.long, device=x.device) for a in idx)
+    return _np(x[tidx])
+
+
+def _streams(k, v, b, hk, n: int):
+    """Gather the distinct (batch, kv-head) key/value streams the rows need.
+
+    Only the first ``n`` rows of each needed stream are copied to the host, so
+    sampled rows of a large device-resident cache stay cheap.
+    """
+    pairs = np.stack([b, hk], axis=1)
+    uniq, inv = np.unique(pairs, axis=0, return_inverse=True)
+    n = max(n, 1)
+    ks = np.stack([_f64(k[int(pb), :n, int(ph), :]) for pb, ph in uniq]) if len(uniq) else \
+        np.zeros((0, n, k.shape[-1]))
+    vs = np.stack([_f64(v[int(pb), :n, int(ph), :]) for pb, ph in uniq]) if len(uniq) else \
+        np.zeros((0, n, v.shape[-1]))
+    return inv.reshape(-1), ks, vs
+
+
+_default: Optional[Oracle] = None
+
+
+def get() -> Oracle:
+    """The oracle built from ``plx_oracle.c`` (compiled on first use if needed)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def prefill(*args, **kw):
+    return get().prefill(*args, **kw)
+
+
+def decode(*args, **kw):
+    return get().decode(*args, **kw)
+
+
+def rows(*args, **kw):
+    return get().rows(*args, **kw)
