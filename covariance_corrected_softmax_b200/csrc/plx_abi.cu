@@ -1,0 +1,260 @@
+// plx_abi.cu -- the C ABI of libplx (declared in include/plx.h): host-side
+// argument checks, TMA descriptor encoding and kernel launches.  No allocation,
+// no synchronisation on the launch paths.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "plx.h"
+#include "plx_launch.h"
+
+
+// The device error word (one per device context); kernels receive its address.
+__device__ unsigned plx_g_device_error = 0;
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_encode_once;
+plx::EncodeTiledFn g_encode = nullptr;
+int g_sm_count[kMaxDevices] = {0};
+unsigned* g_err_ptr[kMaxDevices] = {nullptr};
+std::mutex g_dev_mu;
+
+plx_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return PLX_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device facts: SM count and the device address of the error word.
+cudaError_t device_info(int* sms, unsigned** err) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, plx_g_device_error);
+    if (e != cudaSuccess) return e;
+    g_err_ptr[dev] = static_cast<unsigned*>(ptr);
+    g_sm_count[dev] = n;
+  }
+  if (sms) *sms = g_sm_count[dev];
+  if (err) *err = g_err_ptr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<plx::EncodeTiledFn>(fn);
+  });
+  return g_encode ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// 4-D map over a [B, S, H, D] tensor, box (D, 1, box_rows, 1), no swizzle.
+cudaError_t encode_rows_map(CUtensorMap* map, const void* base, bool bf16, int B, int S, int H,
+                            int D, int box_rows) {
+  cudaError_t e = get_encoder();
+  if (e != cudaSuccess) return e;
+  const cuuint64_t esz = bf16 ? 2 : 4;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {D * esz, (cuuint64_t)H * D * esz, (cuuint64_t)S * H * D * esz};
+  cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        4, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Query heads handled together per pass over a KV head's cache (register
+// budget: two heads' q, rho, o and u per lane).
+int heads_per_pass(int G) { return (G % 2 == 0) ? 2 : 1; }
+
+size_t decode_ws_bytes_for(int d, int hpw, int grid) {
+  const int pf = (d == 64) ? plx::part_floats<64>(hpw) : plx::part_floats<128>(hpw);
+  return (size_t)(plx::kWsHeaderFloats + (size_t)2 * grid * pf) * sizeof(float);
+}
+
+bool shape_ok(int H_q, int H_kv, int d) {
+  return H_q >= 1 && H_kv >= 1 && H_q % H_kv == 0 && (d == 64 || d == 128);
+}
+
+}  // namespace
+
+namespace plx {
+EncodeTiledFn tensor_map_encoder() { return get_encoder() == cudaSuccess ? g_encode : nullptr; }
+}  // namespace plx
+
+extern "C" {
+
+const char* plx_status_string(plx_status s) {
+  switch (s) {
+    case PLX_OK: return "PLX_OK";
+    case PLX_ERR_INVALID_ARGUMENT: return "PLX_ERR_INVALID_ARGUMENT";
+    case PLX_ERR_UNSUPPORTED: return "PLX_ERR_UNSUPPORTED";
+    case PLX_ERR_WORKSPACE_TOO_SMALL: return "PLX_ERR_WORKSPACE_TOO_SMALL";
+    case PLX_ERR_CUDA: return "PLX_ERR_CUDA";
+  }
+  return "PLX_ERR_UNKNOWN";
+}
+
+int plx_last_cuda_error(void) { return t_last_cuda_error; }
+
+int plx_version(void) { return 100; }
+
+plx_status plx_device_error(int* code, int clear) {
+  if (!code) return PLX_ERR_INVALID_ARGUMENT;
+  unsigned v = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemcpyFromSymbol(&v, plx_g_device_error, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (clear) {
+    unsigned z = 0;
+    e = cudaMemcpyToSymbol(plx_g_device_error, &z, sizeof(z));
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  *code = static_cast<int>(v);
+  return PLX_OK;
+}
+
+size_t plx_decode_workspace_bytes(int B, int H_q, int H_kv, int d, int S_max) {
+  if (B < 0 || S_max < 1 || !shape_ok(H_q, H_kv, d)) return 0;
+  int sms = 0;
+  if (device_info(&sms, nullptr) != cudaSuccess) return 0;
+  return decode_ws_bytes_for(d, heads_per_pass(H_q / H_kv), sms);
+}
+
+plx_status plx_decode(const void* q, const void* rho, const void* k_cache, const void* v_cache,
+                      const int32_t* seqlens, void* out, int B, int H_q, int H_kv, int d,
+                      int S_max, plx_dtype dtype, float softmax_scale, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  t_last_cuda_error = 0;
+  if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
+  if (B < 0 || S_max < 1 || !shape_ok(H_q, H_kv, d)) return PLX_ERR_INVALID_ARGUMENT;
+  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (B == 0) return PLX_OK;
+  if (!q || !rho || !k_cache || !v_cache || !seqlens || !out || !workspace)
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(rho) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(out) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return PLX_ERR_INVALID_ARGUMENT;
+  // TMA coordinates are 32-bit; cache extents must fit.
+  if ((long long)B * S_max > (1ll << 31) || (long long)B * H_q > (1 << 30))
+    return PLX_ERR_UNSUPPORTED;
+
+  const bool bf16 = dtype == PLX_BF16;
+  const int G = H_q / H_kv;
+  const int hpw = heads_per_pass(G);
+  int sms = 0;
+  unsigned* err = nullptr;
+  cudaError_t e = device_info(&sms, &err);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int tk = plx::decode_tile_keys(bf16, d);
+  const long long max_tiles = (long long)B * H_kv * (G / hpw) * ((S_max + tk - 1) / tk);
+  const int grid = (int)(max_tiles < sms ? max_tiles : sms);
+  if (workspace_bytes < decode_ws_bytes_for(d, hpw, sms)) return PLX_ERR_WORKSPACE_TOO_SMALL;
+
+  CUtensorMap kmap, vmap;
+  e = encode_rows_map(&kmap, k_cache, bf16, B, S_max, H_kv, d, tk);
+  if (e == cudaSuccess) e = encode_rows_map(&vmap, v_cache, bf16, B, S_max, H_kv, d, tk);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  plx::DecodeParams p;
+  p.q = q;
+  p.rho = rho;
+  p.seqlens = seqlens;
+  p.out = out;
+  p.ws = static_cast<float*>(workspace);
+  p.B = B;
+  p.Hq = H_q;
+  p.Hkv = H_kv;
+  p.G = G;
+  p.S_max = S_max;
+  p.nhg = G / hpw;
+  p.qscale = softmax_scale * 1.4426950408889634f;
+  p.grid = grid;
+  p.err = err;
+  e = plx::launch_decode(bf16, d, kmap, vmap, p, hpw, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return PLX_OK;
+}
+
+plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k, const void* v,
+                           void* out, float* lse, int causal, int B, int L, int H_q, int H_kv,
+                           int d, plx_dtype dtype, float softmax_scale, void* stream) {
+  t_last_cuda_error = 0;
+  if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
+  if (B < 0 || L < 0 || !shape_ok(H_q, H_kv, d) || (causal != 0 && causal != 1))
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (B == 0 || L == 0) return PLX_OK;
+  if (!q || !rho || !k || !v || !out) return PLX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(rho) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return PLX_ERR_INVALID_ARGUMENT;
+  if ((long long)B * L > (1ll << 31) || B > 65535 || H_q > 65535) return PLX_ERR_UNSUPPORTED;
+
+  int sms = 0;
+  unsigned* err = nullptr;
+  cudaError_t e = device_info(&sms, &err);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PLX_F32) {
+    plx::PrefillSimtParams p;
+    p.q = static_cast<const float*>(q);
+    p.rho = static_cast<const float*>(rho);
+    p.k = static_cast<const float*>(k);
+    p.v = static_cast<const float*>(v);
+    p.out = static_cast<float*>(out);
+    p.lse = lse;
+    p.B = B;
+    p.L = L;
+    p.Hq = H_q;
+    p.Hkv = H_kv;
+    p.G = H_q / H_kv;
+    p.causal = causal;
+    p.scale = softmax_scale;
+    e = plx::launch_prefill_simt(p, d, st);
+    return e == cudaSuccess ? PLX_OK : cuda_fail(e);
+  }
+  plx::PrefillTcArgs a;
+  a.q = q;
+  a.rho = rho;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.lse = lse;
+  a.B = B;
+  a.L = L;
+  a.Hq = H_q;
+  a.Hkv = H_kv;
+  a.d = d;
+  a.causal = causal;
+  a.scale = softmax_scale;
+  a.err = err;
+  a.num_sms = sms;
+  e = plx::launch_prefill_tc(a, st);
+  if (e == cudaErrorNotSupported) return PLX_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? PLX_OK : cuda_fail(e);
+}
+
+}  // extern "C"

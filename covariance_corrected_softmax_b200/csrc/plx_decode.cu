@@ -1,0 +1,580 @@
+// plx_decode.cu -- Parallax decode kernels: persistent split-K main kernel and
+// the log-sum-exp combine kernel.  See plx_decode.cuh for the design.
+#include "plx_launch.h"
+
+namespace plx {
+
+// ---------------------------------------------------------------------------
+// Element helpers: EPL consecutive elements -> EPL/2 float2.
+// ---------------------------------------------------------------------------
+template <typename T, int EPL>
+struct RowLoad;
+
+template <int EPL>
+struct RowLoad<__nv_bfloat16, EPL> {
+  static_assert(EPL == 4 || EPL == 8, "bf16 lane slice is 8 or 16 bytes");
+  __device__ __forceinline__ static void load(const void* p, float2 (&f)[EPL / 2]) {
+    if constexpr (EPL == 8) {
+      uint4 w = *reinterpret_cast<const uint4*>(p);
+      f[0] = bf16x2_to_float2(w.x);
+      f[1] = bf16x2_to_float2(w.y);
+      f[2] = bf16x2_to_float2(w.z);
+      f[3] = bf16x2_to_float2(w.w);
+    } else {
+      uint2 w = *reinterpret_cast<const uint2*>(p);
+      f[0] = bf16x2_to_float2(w.x);
+      f[1] = bf16x2_to_float2(w.y);
+    }
+  }
+};
+
+template <int EPL>
+struct RowLoad<float, EPL> {
+  static_assert(EPL == 4 || EPL == 8, "fp32 lane slice is 16 or 32 bytes");
+  __device__ __forceinline__ static void load(const void* p, float2 (&f)[EPL / 2]) {
+    const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+    for (int i = 0; i < EPL / 4; ++i) {
+      float4 w = q[i];
+      f[2 * i] = make_float2(w.x, w.y);
+      f[2 * i + 1] = make_float2(w.z, w.w);
+    }
+  }
+};
+
+template <typename T>
+__device__ __forceinline__ void store_elem(void* out, size_t idx, float x);
+template <>
+__device__ __forceinline__ void store_elem<__nv_bfloat16>(void* out, size_t idx, float x) {
+  reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ void store_elem<float>(void* out, size_t idx, float x) {
+  reinterpret_cast<float*>(out)[idx] = x;
+}
+
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// exp2 of (x - m) where x may be -inf; m = -inf only when every x is -inf.
+__device__ __forceinline__ float exp2_shift(float x, float m) {
+  return (m == -INFINITY) ? 0.f : exp2f(x - m);
+}
+
+// Combine weight exp2(m - M) of a partial state with running max m into a
+// merged state with max M >= m (0 for an empty state).
+__device__ __forceinline__ float merge_weight(float m, float M) {
+  return (m == -INFINITY) ? 0.f : exp2f(m - M);
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide search for this CTA's tile range.  Tiles are ordered batch-major;
+// batch b holds ceil(len_b / TK) tiles for each of its Hkv * nhg segments.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ long long batch_tiles(const int32_t* seqlens, int b, int S_max,
+                                                 int TK, int segs_per_b) {
+  int len = clamp_len(seqlens[b], S_max);
+  return (long long)((len + TK - 1) / TK) * segs_per_b;
+}
+
+struct RangeInfo {
+  long long total, t0, t1;
+  int b0;              // batch holding tile t0 (valid when t0 < t1)
+  long long off0;      // t0 minus the first tile of batch b0
+};
+
+__device__ void locate_range(const DecodeParams& p, int TK, RangeInfo* info, long long* scan_ws) {
+  const int tid = threadIdx.x, nth = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarps = nth >> 5;
+  const int segs_per_b = p.Hkv * p.nhg;
+  const int per = (p.B + nth - 1) / nth;
+  const int lo = min(p.B, tid * per), hi = min(p.B, lo + per);
+  long long local = 0;
+  for (int b = lo; b < hi; ++b) local += batch_tiles(p.seqlens, b, p.S_max, TK, segs_per_b);
+  // inclusive warp scan
+  long long inc = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    long long y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) scan_ws[warp] = inc;
+  __syncthreads();
+  if (tid == 0) {
+    long long run = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      long long x = scan_ws[w];
+      scan_ws[w] = run;
+      run += x;
+    }
+    scan_ws[nwarps] = run;
+  }
+  __syncthreads();
+  const long long excl = scan_ws[warp] + inc - local;
+  const long long total = scan_ws[nwarps];
+  const long long t0 = total * blockIdx.x / p.grid;
+  const long long t1 = total * (blockIdx.x + 1) / p.grid;
+  if (tid == 0) {
+    info->total = total;
+    info->t0 = t0;
+    info->t1 = t1;
+    info->b0 = -1;
+    info->off0 = 0;
+  }
+  __syncthreads();
+  if (t0 < t1 && excl <= t0 && t0 < excl + local) {
+    long long run = excl;
+    for (int b = lo; b < hi; ++b) {
+      long long c = batch_tiles(p.seqlens, b, p.S_max, TK, segs_per_b);
+      if (t0 < run + c) {
+        info->b0 = b;
+        info->off0 = t0 - run;
+        break;
+      }
+      run += c;
+    }
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// Main decode kernel.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int HPW>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    plx_decode_splitk_kernel(const __grid_constant__ CUtensorMap kmap,
+                             const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+  using Cfg = DecodeTile<T, D>;
+  constexpr int TK = Cfg::TK, KPH = Cfg::KPH, EPL = Cfg::EPL, STAGES = Cfg::STAGES;
+  constexpr int H2 = EPL / 2;
+  constexpr int PF = part_floats<D>(HPW);
+  constexpr int PHF = part_head_floats<D>();
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  TileMeta* metas = reinterpret_cast<TileMeta*>(ring + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(metas + STAGES);
+  uint64_t* empty = full + STAGES;
+  RangeInfo* info = reinterpret_cast<RangeInfo*>(empty + STAGES);
+  long long* scan_ws = reinterpret_cast<long long*>(info + 1);   // 16 entries
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(scan_ws + 16);
+  float* merge = reinterpret_cast<float*>(scan_ws + 20);          // 16-byte aligned
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    *abort_flag = 0;
+    // Invalidate this CTA's two partial slots; finalisation rewrites them.
+    int* s0 = reinterpret_cast<int*>(p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x) * PF);
+    int* s1 = reinterpret_cast<int*>(p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + 1) * PF);
+    s0[0] = -1;
+    s1[0] = -1;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDecConsumerWarps);
+    }
+    fence_mbarrier_init();
+  }
+  locate_range(p, TK, info, scan_ws);  // contains __syncthreads
+  if (blockIdx.x == 0 && tid == 0) reinterpret_cast<long long*>(p.ws)[0] = info->total;
+
+  // Batches with an empty context produce zeros (out = 0 for an empty key set).
+  for (int b = blockIdx.x; b < p.B; b += p.grid) {
+    if (clamp_len(p.seqlens[b], p.S_max) == 0) {
+      for (int e = tid; e < p.Hq * D; e += blockDim.x)
+        store_elem<T>(p.out, (size_t)b * p.Hq * D + e, 0.f);
+    }
+  }
+
+  const long long t0 = info->t0, t1 = info->t1;
+  const int segs_per_b = p.Hkv * p.nhg;
+
+  if (warp == kDecConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && t0 < t1) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      int b = info->b0;
+      int len = clamp_len(p.seqlens[b], p.S_max);
+      int nt = (len + TK - 1) / TK;
+      int seg_local = (int)(info->off0 / nt);
+      int kt = (int)(info->off0 % nt);
+      bool starts_here = (kt == 0);
+      for (long long t = t0, i = 0; t < t1; ++t, ++i) {
+        const int stage = (int)(i % STAGES);
+        if (i >= STAGES) {
+          if (!mbar_wait(&empty[stage], (uint32_t)(((i / STAGES) - 1) & 1), abort_flag, p.err)) break;
+        }
+        TileMeta m;
+        m.b = b;
+        m.hkv = seg_local / p.nhg;
+        m.hg = seg_local % p.nhg;
+        m.kt = kt;
+        m.nvalid = min(TK, len - kt * TK);
+        m.seg = b * segs_per_b + seg_local;
+        m.flags = ((t == t0 || kt == 0) ? 1 : 0) | ((t == t1 - 1 || kt == nt - 1) ? 2 : 0) |
+                  (starts_here ? 4 : 0) | ((kt == nt - 1) ? 8 : 0);
+        m.pad = 0;
+        metas[stage] = m;
+        mbar_arrive_expect_tx(&full[stage], 2 * Cfg::TILE_BYTES);
+        uint8_t* dst = ring + stage * Cfg::STAGE_BYTES;
+        tma_load_4d(dst, &kmap, &full[stage], 0, m.hkv, kt * TK, b);
+        tma_load_4d(dst + Cfg::TILE_BYTES, &vmap, &full[stage], 0, m.hkv, kt * TK, b);
+        // advance the walk
+        if (++kt == nt) {
+          kt = 0;
+          starts_here = true;
+          if (++seg_local == segs_per_b) {
+            seg_local = 0;
+            do {
+              ++b;
+            } while (b < p.B && clamp_len(p.seqlens[b], p.S_max) == 0);
+            if (b < p.B) {
+              len = clamp_len(p.seqlens[b], p.S_max);
+              nt = (len + TK - 1) / TK;
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int hw = lane >> 4, sub = lane & 15;
+    const int rowbase = (warp * 2 + hw) * KPH;
+    float2 qf[HPW][H2], rf[HPW][H2], oa[HPW][H2], ua[HPW][H2];
+    float m[HPW], l[HPW], z[HPW];
+    int ordinal = 0;
+#pragma unroll
+    for (int g = 0; g < HPW; ++g) {
+      m[g] = -INFINITY;
+      l[g] = 0.f;
+      z[g] = 0.f;
+#pragma unroll
+      for (int e = 0; e < H2; ++e) {
+        qf[g][e] = rf[g][e] = oa[g][e] = ua[g][e] = make_float2(0.f, 0.f);
+      }
+    }
+
+    for (long long t = t0, i = 0; t < t1; ++t, ++i) {
+      const int stage = (int)(i % STAGES);
+      if (!mbar_wait(&full[stage], (uint32_t)((i / STAGES) & 1), abort_flag, p.err)) break;
+      const TileMeta mt = metas[stage];
+      const int h0 = mt.hkv * p.G + mt.hg * HPW;  // first query head of the group
+
+      if (mt.flags & 1) {  // first tile of a segment in this CTA: load q, rho; reset
+#pragma unroll
+        for (int g = 0; g < HPW; ++g) {
+          const size_t base = ((size_t)mt.b * p.Hq + h0 + g) * D + sub * EPL;
+          RowLoad<T, EPL>::load(reinterpret_cast<const T*>(p.q) + base, qf[g]);
+          RowLoad<T, EPL>::load(reinterpret_cast<const T*>(p.rho) + base, rf[g]);
+#pragma unroll
+          for (int e = 0; e < H2; ++e) {
+            qf[g][e].x *= p.qscale;
+            qf[g][e].y *= p.qscale;
+            oa[g][e] = ua[g][e] = make_float2(0.f, 0.f);
+          }
+          m[g] = -INFINITY;
+          l[g] = 0.f;
+          z[g] = 0.f;
+        }
+      }
+
+      const uint8_t* kt_base = ring + stage * Cfg::STAGE_BYTES +
+                               (size_t)rowbase * Cfg::ROW_BYTES + sub * EPL * sizeof(T);
+      const uint8_t* vt_base = kt_base + Cfg::TILE_BYTES;
+
+      // Phase A: partial dot products s = (scale log2e) q.k and t = rho.k
+      float s[KPH][HPW], tt[KPH][HPW];
+#pragma unroll
+      for (int kk = 0; kk < KPH; ++kk) {
+        float2 kf[H2];
+        RowLoad<T, EPL>::load(kt_base + kk * Cfg::ROW_BYTES, kf);
+#pragma unroll
+        for (int g = 0; g < HPW; ++g) {
+          float2 as = make_float2(0.f, 0.f), at = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int e = 0; e < H2; ++e) {
+            as = __ffma2_rn(qf[g][e], kf[e], as);
+            at = __ffma2_rn(rf[g][e], kf[e], at);
+          }
+          s[kk][g] = as.x + as.y;
+          tt[kk][g] = at.x + at.y;
+        }
+      }
+      // Phase B: reduce over the 16 lanes of the half-warp
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) {
+#pragma unroll
+        for (int kk = 0; kk < KPH; ++kk) {
+#pragma unroll
+          for (int g = 0; g < HPW; ++g) {
+            s[kk][g] += __shfl_xor_sync(0xffffffffu, s[kk][g], off);
+            tt[kk][g] += __shfl_xor_sync(0xffffffffu, tt[kk][g], off);
+          }
+        }
+      }
+      // Phase C: online softmax over this half-warp's KPH keys
+      bool valid[KPH];
+#pragma unroll
+      for (int kk = 0; kk < KPH; ++kk) valid[kk] = (rowbase + kk) < mt.nvalid;
+      float pw[KPH][HPW], ptw[KPH][HPW];
+#pragma unroll
+      for (int g = 0; g < HPW; ++g) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int kk = 0; kk < KPH; ++kk) {
+          if (!valid[kk]) s[kk][g] = -INFINITY;
+          mx = fmaxf(mx, s[kk][g]);
+        }
+        if (mx > m[g]) {
+          const float alpha = merge_weight(m[g], mx);
+          l[g] *= alpha;
+          z[g] *= alpha;
+#pragma unroll
+          for (int e = 0; e < H2; ++e) {
+            oa[g][e] = __fmul2_rn(oa[g][e], f2(alpha));
+            ua[g][e] = __fmul2_rn(ua[g][e], f2(alpha));
+          }
+          m[g] = mx;
+        }
+#pragma unroll
+        for (int kk = 0; kk < KPH; ++kk) {
+          const float pr = exp2_shift(s[kk][g], m[g]);
+          const float pt = pr * tt[kk][g];
+          pw[kk][g] = pr;
+          ptw[kk][g] = valid[kk] ? pt : 0.f;
+          l[g] += pr;
+          z[g] += ptw[kk][g];
+        }
+      }
+      // Phase D: accumulate o += p v and u += (p t) v
+#pragma unroll
+      for (int kk = 0; kk < KPH; ++kk) {
+        float2 vf[H2];
+        RowLoad<T, EPL>::load(vt_base + kk * Cfg::ROW_BYTES, vf);
+        if (!valid[kk]) {
+#pragma unroll
+          for (int e = 0; e < H2; ++e) vf[e] = make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int g = 0; g < HPW; ++g) {
+#pragma unroll
+          for (int e = 0; e < H2; ++e) {
+            oa[g][e] = __ffma2_rn(f2(pw[kk][g]), vf[e], oa[g][e]);
+            ua[g][e] = __ffma2_rn(f2(ptw[kk][g]), vf[e], ua[g][e]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+
+      if (mt.flags & 2) {
+        // ---- finalise the segment: merge the 16 half-warp states
+#pragma unroll
+        for (int g = 0; g < HPW; ++g) {
+          const float mo = __shfl_xor_sync(0xffffffffu, m[g], 16);
+          const float M = fmaxf(m[g], mo);
+          const float w = merge_weight(m[g], M);
+          float lw = l[g] * w, zw = z[g] * w;
+          lw += __shfl_xor_sync(0xffffffffu, lw, 16);
+          zw += __shfl_xor_sync(0xffffffffu, zw, 16);
+          m[g] = M;
+          l[g] = lw;
+          z[g] = zw;
+#pragma unroll
+          for (int e = 0; e < H2; ++e) {
+            float2 ow = __fmul2_rn(oa[g][e], f2(w)), uw = __fmul2_rn(ua[g][e], f2(w));
+            ow.x += __shfl_xor_sync(0xffffffffu, ow.x, 16);
+            ow.y += __shfl_xor_sync(0xffffffffu, ow.y, 16);
+            uw.x += __shfl_xor_sync(0xffffffffu, uw.x, 16);
+            uw.y += __shfl_xor_sync(0xffffffffu, uw.y, 16);
+            oa[g][e] = ow;
+            ua[g][e] = uw;
+          }
+          if (hw == 0) {
+            float* dst = merge + (warp * HPW + g) * PHF;
+            if (sub == 0) {
+              dst[0] = M;
+              dst[1] = lw;
+              dst[2] = zw;
+            }
+#pragma unroll
+            for (int e = 0; e < H2; ++e) {
+              dst[4 + sub * EPL + 2 * e] = oa[g][e].x;
+              dst[4 + sub * EPL + 2 * e + 1] = oa[g][e].y;
+              dst[4 + D + sub * EPL + 2 * e] = ua[g][e].x;
+              dst[4 + D + sub * EPL + 2 * e + 1] = ua[g][e].y;
+            }
+          }
+        }
+        named_bar_sync(1, kDecConsumerWarps * 32);
+        const bool complete = (mt.flags & 4) && (mt.flags & 8);
+        const int slot = ordinal == 0 ? 0 : 1;
+        float* part = p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + slot) * PF;
+        for (int pr = tid; pr < HPW * D; pr += kDecConsumerWarps * 32) {
+          const int g = pr / D, c = pr % D;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, merge[(w * HPW + g) * PHF]);
+          float L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
+#pragma unroll
+          for (int w = 0; w < kDecConsumerWarps; ++w) {
+            const float* src = merge + (w * HPW + g) * PHF;
+            const float wt = merge_weight(src[0], M);
+            L += wt * src[1];
+            Z += wt * src[2];
+            O += wt * src[4 + c];
+            U += wt * src[4 + D + c];
+          }
+          if (complete) {
+            // out = (1 + tbar) o - u with tbar = Z/L, o = O/L, u = U/L
+            const float inv = 1.f / L;
+            const float val = ((1.f + Z * inv) * O - U) * inv;
+            store_elem<T>(p.out, ((size_t)mt.b * p.Hq + h0 + g) * D + c, val);
+          } else {
+            float* ph = part + kPartHeader + g * PHF;
+            if (c == 0) {
+              ph[0] = M;
+              ph[1] = L;
+              ph[2] = Z;
+            }
+            ph[4 + c] = O;
+            ph[4 + D + c] = U;
+          }
+        }
+        if (!complete && tid == 0) {
+          int* hdr = reinterpret_cast<int*>(part);
+          hdr[1] = (mt.flags & 4) ? 1 : 0;
+          hdr[2] = (mt.flags & 8) ? 1 : 0;
+          hdr[3] = 0;
+          hdr[0] = mt.seg;
+        }
+        named_bar_sync(1, kDecConsumerWarps * 32);
+        ++ordinal;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Combine kernel: one block per main-kernel CTA.  A block whose CTA holds the
+// head piece of a split segment merges that segment's pieces (the head piece,
+// then the first slot of each following CTA until the piece that ends it).
+// ---------------------------------------------------------------------------
+template <typename T, int D, int HPW>
+__global__ void __launch_bounds__(256)
+    plx_decode_combine_kernel(const DecodeParams p) {
+  constexpr int PF = part_floats<D>(HPW);
+  constexpr int PHF = part_head_floats<D>();
+  const float* base = p.ws + kWsHeaderFloats;
+  const int c0 = blockIdx.x;
+  int slot = -1;
+  for (int s = 1; s >= 0; --s) {
+    const int* hdr = reinterpret_cast<const int*>(base + (size_t)(2 * c0 + s) * PF);
+    if (hdr[0] >= 0 && hdr[1] == 1) {
+      slot = s;
+      break;
+    }
+  }
+  if (slot < 0) return;
+  const int* hdr0 = reinterpret_cast<const int*>(base + (size_t)(2 * c0 + slot) * PF);
+  const int seg = hdr0[0];
+  const int segs_per_b = p.Hkv * p.nhg;
+  const int b = seg / segs_per_b, seg_local = seg % segs_per_b;
+  const int hkv = seg_local / p.nhg, hg = seg_local % p.nhg;
+  const int h0 = hkv * p.G + hg * HPW;
+
+  for (int pr = threadIdx.x; pr < HPW * D; pr += blockDim.x) {
+    const int g = pr / D, c = pr % D;
+    float M = -INFINITY, L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
+    int cta = c0, s = slot;
+    bool ok = false;
+    while (cta < p.grid) {
+      const float* piece = base + (size_t)(2 * cta + s) * PF;
+      const int* hdr = reinterpret_cast<const int*>(piece);
+      if (hdr[0] == seg) {
+        const float* ph = piece + kPartHeader + g * PHF;
+        const float m = ph[0];
+        const float Mn = fmaxf(M, m);
+        const float wa = merge_weight(M, Mn), wb = merge_weight(m, Mn);
+        L = L * wa + ph[1] * wb;
+        Z = Z * wa + ph[2] * wb;
+        O = O * wa + ph[4 + c] * wb;
+        U = U * wa + ph[4 + D + c] * wb;
+        M = Mn;
+        if (hdr[2] == 1) {
+          ok = true;
+          break;
+        }
+      } else if (hdr[0] != -1 || cta == c0) {
+        // Tiles are contiguous: between two pieces of a segment there can only
+        // be CTAs that received no tiles at all (both slots invalid).
+        break;
+      }
+      ++cta;
+      s = 0;
+    }
+    if (!ok) {
+      record_error(p.err, kDevBadArgument);
+      continue;
+    }
+    const float inv = 1.f / L;
+    const float val = ((1.f + Z * inv) * O - U) * inv;
+    store_elem<T>(p.out, ((size_t)b * p.Hq + h0 + g) * D + c, val);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launch helpers (called from plx_abi.cu).
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+constexpr int decode_smem_bytes(int hpw) {
+  using Cfg = DecodeTile<T, D>;
+  return 1024 + Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::STAGES * (int)sizeof(TileMeta) +
+         2 * Cfg::STAGES * 8 + (int)sizeof(RangeInfo) + 20 * 8 +
+         kDecConsumerWarps * hpw * part_head_floats<D>() * 4;
+}
+
+template <typename T, int D, int HPW>
+cudaError_t launch_decode_t(const CUtensorMap& kmap, const CUtensorMap& vmap,
+                            const DecodeParams& p, cudaStream_t stream) {
+  const int smem = decode_smem_bytes<T, D>(HPW);
+  auto kern = plx_decode_splitk_kernel<T, D, HPW>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<p.grid, kDecThreads, smem, stream>>>(kmap, vmap, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  plx_decode_combine_kernel<T, D, HPW><<<p.grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_decode_d(const CUtensorMap& kmap, const CUtensorMap& vmap,
+                            const DecodeParams& p, int hpw, cudaStream_t stream) {
+  switch (hpw) {
+    case 1: return launch_decode_t<T, D, 1>(kmap, vmap, p, stream);
+    case 2: return launch_decode_t<T, D, 2>(kmap, vmap, p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_decode(bool bf16, int d, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                          const DecodeParams& p, int hpw, cudaStream_t stream) {
+  if (bf16) {
+    if (d == 64) return launch_decode_d<__nv_bfloat16, 64>(kmap, vmap, p, hpw, stream);
+    if (d == 128) return launch_decode_d<__nv_bfloat16, 128>(kmap, vmap, p, hpw, stream);
+  } else {
+    if (d == 64) return launch_decode_d<float, 64>(kmap, vmap, p, hpw, stream);
+    if (d == 128) return launch_decode_d<float, 128>(kmap, vmap, p, hpw, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+int decode_tile_keys(bool bf16, int d) {
+  (void)d;
+  return bf16 ? DecodeTile<__nv_bfloat16, 128>::TK : DecodeTile<float, 128>::TK;
+}
+
+}  // namespace plx

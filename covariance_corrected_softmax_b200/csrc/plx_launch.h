@@ -1,0 +1,52 @@
+// plx_launch.h -- host-side declarations shared by the ABI layer and the
+// kernel files: launch parameter structs and launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "plx_decode.cuh"
+
+namespace plx {
+
+struct PrefillSimtParams {
+  const float* q;    // [B, L, Hq, D]
+  const float* rho;  // [B, L, Hq, D]
+  const float* k;    // [B, L, Hkv, D]
+  const float* v;    // [B, L, Hkv, D]
+  float* out;        // [B, L, Hq, D]
+  float* lse;        // [B, Hq, L] or null
+  int B, L, Hq, Hkv, G, causal;
+  float scale;
+};
+
+struct PrefillTcArgs {
+  const void* q;
+  const void* rho;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;
+  int B, L, Hq, Hkv, d, causal;
+  float scale;
+  unsigned* err;
+  int num_sms;
+};
+
+cudaError_t launch_prefill_simt(const PrefillSimtParams& p, int d, cudaStream_t stream);
+// Tensor-core (tcgen05) bf16 prefill; encodes its own TMA descriptors.
+cudaError_t launch_prefill_tc(const PrefillTcArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(bool bf16, int d, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                          const DecodeParams& p, int hpw, cudaStream_t stream);
+int decode_tile_keys(bool bf16, int d);
+
+// TMA descriptor encoder (cuTensorMapEncodeTiled through the runtime's driver
+// entry point); null if unavailable.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
+
+}  // namespace plx

@@ -1,0 +1,169 @@
+"""Thin ctypes binding of libplx (the C ABI in include/plx.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  PyTorch supplies device memory (outputs, decode
+workspace) and the current CUDA stream.  There is no fallback: if the library
+is missing or a call fails, these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libplx.so")
+
+PLX_OK, PLX_ERR_INVALID_ARGUMENT, PLX_ERR_UNSUPPORTED, PLX_ERR_WORKSPACE_TOO_SMALL, \
+    PLX_ERR_CUDA = range(5)
+PLX_F32, PLX_BF16 = 0, 1
+_DTYPES = {torch.float32: PLX_F32, torch.bfloat16: PLX_BF16}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class PlxError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = f"{what}: {status_string(status)}"
+        if status == PLX_ERR_CUDA:
+            msg += f" (cudaError {lib().plx_last_cuda_error()})"
+        super().__init__(msg)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libplx.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m covariance_corrected_softmax_b200.build` (or __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.plx_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp]
+        L.plx_prefill_fwd.restype = i
+        L.plx_decode_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.plx_decode_workspace_bytes.restype = sz
+        L.plx_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, sz, vp]
+        L.plx_decode.restype = i
+        L.plx_status_string.argtypes = [i]
+        L.plx_status_string.restype = ctypes.c_char_p
+        L.plx_last_cuda_error.argtypes = []
+        L.plx_last_cuda_error.restype = i
+        L.plx_device_error.argtypes = [ctypes.POINTER(i), i]
+        L.plx_device_error.restype = i
+        L.plx_version.argtypes = []
+        L.plx_version.restype = i
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().plx_status_string(status).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != PLX_OK:
+        raise PlxError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+    return _DTYPES[t.dtype]
+
+
+def _same(ref: torch.Tensor, *ts: torch.Tensor) -> None:
+    for t in ts:
+        if t.dtype != ref.dtype or t.device != ref.device:
+            raise TypeError("q, rho, k and v must share dtype and device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def prefill(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+            causal: bool = True, softmax_scale: Optional[float] = None,
+            return_lse: bool = True, out: Optional[torch.Tensor] = None,
+            lse: Optional[torch.Tensor] = None, stream=None
+            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Parallax attention forward: q, rho [B, L, Hq, d]; k, v [B, L, Hkv, d].
+
+    Returns (out [B, L, Hq, d], lse [B, Hq, L] fp32 or None).  softmax_scale
+    defaults to 1/sqrt(d).
+    """
+    _same(q, rho, k, v)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if rho.shape != q.shape or k.shape != (B, L, Hkv, d) or v.shape != k.shape:
+        raise ValueError("shape mismatch among q, rho, k, v")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    st = lib().plx_prefill_fwd(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out),
+                               _ptr(lse) if return_lse else None, int(bool(causal)), B, L, Hq,
+                               Hkv, d, _dtype_code(q), scale, _stream(stream))
+    _check(st, "plx_prefill_fwd")
+    return out, (lse if return_lse else None)
+
+
+def decode_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, S_max: int) -> int:
+    return int(lib().plx_decode_workspace_bytes(B, Hq, Hkv, d, S_max))
+
+
+def decode_workspace(B: int, Hq: int, Hkv: int, d: int, S_max: int,
+                     device=None) -> torch.Tensor:
+    """A device buffer sized for plx_decode on the current device."""
+    n = decode_workspace_bytes(B, Hq, Hkv, d, S_max)
+    if n == 0:
+        raise ValueError("invalid decode shape")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def decode(q: torch.Tensor, rho: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+           seqlens: torch.Tensor, softmax_scale: Optional[float] = None,
+           out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+           stream=None) -> torch.Tensor:
+    """Single-token decode: q, rho [B, Hq, d]; caches [B, S_max, Hkv, d];
+    seqlens int32 [B] on the device.  Returns out [B, Hq, d]."""
+    _same(q, rho, k_cache, v_cache)
+    B, Hq, d = q.shape
+    S_max, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if rho.shape != q.shape or k_cache.shape != (B, S_max, Hkv, d) or \
+            v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch among q, rho, k_cache, v_cache")
+    if seqlens.dtype != torch.int32 or seqlens.device != q.device or seqlens.numel() != B:
+        raise ValueError("seqlens must be int32 [B] on the same device")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, Hkv, d, S_max, device=q.device)
+    st = lib().plx_decode(_ptr(q), _ptr(rho), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+                          _ptr(out), B, Hq, Hkv, d, S_max, _dtype_code(q), scale,
+                          _ptr(workspace), workspace.numel() * workspace.element_size(),
+                          _stream(stream))
+    _check(st, "plx_decode")
+    return out
+
+
+def device_error(clear: bool = True) -> int:
+    """The kernels' device-side error word (0 = none); synchronises."""
+    code = ctypes.c_int(0)
+    _check(lib().plx_device_error(ctypes.byref(code), int(clear)), "plx_device_error")
+    return code.value

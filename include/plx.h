@@ -1,0 +1,140 @@
+/*
+ * plx.h -- C ABI of libplx: Parallax attention on NVIDIA B200 (sm_100a).
+ *
+ * Parallax (page 1 "Parallax: Parameterized Local Linear Attention Gives
+ * Transformers a 'Second Eye'", opening formula and section 1.3; page 3
+ * "Parallax keeps softmax, adds covariance correction branch") is softmax
+ * attention with an additive covariance correction.  For query row i,
+ *
+ *     out_i = o_SA,i - Sigma_KV^(i)^T rho_i
+ *
+ *     a_ij         = softmax_j(softmax_scale * q_i . k_j)       (page 1, 1.1)
+ *     o_SA,i       = sum_j a_ij v_j
+ *     mu_i         = sum_j a_ij k_j
+ *     Sigma_KV^(i) = sum_j a_ij (k_j - mu_i)(v_j - o_SA,i)^T  (d x d, the
+ *                    softmax-weighted covariance of K and V, page 1, 1.3)
+ *     rho_i        = the probe (W_R x_i in a model; an input here), contracted
+ *                    with the key index of Sigma_KV.
+ *
+ * rho = 0 gives plain softmax attention (page 3: W_R = 0 recovers softmax).
+ * The kernels use the equal one-pass form out = (1 + tbar) o - u with
+ * t_j = rho . k_j, tbar = sum a t, u = sum a t v, so a single pass over K and V
+ * feeds both branches (page 3: the KV stream is reused by both branches).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers, owned by the caller, contiguous,
+ *     row-major in the layouts given below, and 16-byte aligned.  The library
+ *     never allocates, frees or synchronises; it only enqueues work.
+ *   - dtype applies to q, rho, k, v and out alike.  Accumulation is fp32.
+ *     PLX_BF16 runs on the tensor cores (prefill) or streams a bf16 cache
+ *     (decode); PLX_F32 computes every product in fp32 on the CUDA cores.
+ *   - d (head dimension, d_k = d_v) must be 64 or 128; H_q must be a multiple
+ *     of H_kv.  Query head h reads key/value head h / (H_q / H_kv).
+ *   - stream is a cudaStream_t (NULL = the legacy default stream).  Work runs
+ *     asynchronously on it, in order with the caller's other work there.
+ *   - Arguments are checked on the host before anything is enqueued; a bad
+ *     argument returns PLX_ERR_INVALID_ARGUMENT or PLX_ERR_UNSUPPORTED and
+ *     enqueues nothing.  A failed launch returns PLX_ERR_CUDA
+ *     (plx_last_cuda_error() gives the cudaError_t).  Faults during execution
+ *     surface at the caller's next synchronisation; kernels never wait forever:
+ *     a wait that runs out of time records a code readable by
+ *     plx_device_error() and the kernel returns.
+ *   - Thread safety: calls may come from several host threads; the
+ *     per-thread error code is thread-local.
+ */
+#ifndef PLX_H_
+#define PLX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PLX_API __attribute__((visibility("default")))
+#else
+#define PLX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum plx_status {
+  PLX_OK = 0,
+  PLX_ERR_INVALID_ARGUMENT = 1,    /* null/misaligned pointer, bad size      */
+  PLX_ERR_UNSUPPORTED = 2,         /* valid request this build cannot run    */
+  PLX_ERR_WORKSPACE_TOO_SMALL = 3, /* decode workspace below the query size  */
+  PLX_ERR_CUDA = 4                 /* a CUDA runtime call or launch failed   */
+} plx_status;
+
+typedef enum plx_dtype { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
+
+/*
+ * plx_prefill_fwd -- multi-head / grouped-query Parallax attention forward.
+ *
+ *   q, rho : [B, L, H_q, d]   queries and probes (one probe per query row)
+ *   k, v   : [B, L, H_kv, d]  keys and values
+ *   out    : [B, L, H_q, d]   written
+ *   lse    : [B, H_q, L] fp32, written if non-NULL: natural-log
+ *            log-sum-exp of the scaled scores of each row (the softmax
+ *            normaliser; independent of rho)
+ *   causal : 1 = row i sees keys 0..i; 0 = every row sees all L keys
+ *   softmax_scale : the score scale (1/sqrt(d) in the textbook form,
+ *            page 1 section 1.1); any finite value
+ * Sizes: B, L, H_q, H_kv >= 1 (B == 0 or L == 0 is a no-op returning PLX_OK).
+ * Operator definition: page 1 section 1.3 and page 3 (see the file header).
+ */
+PLX_API plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k, const void* v,
+                           void* out, float* lse, int causal, int B, int L, int H_q,
+                           int H_kv, int d, plx_dtype dtype, float softmax_scale,
+                           void* stream);
+
+/*
+ * plx_decode_workspace_bytes -- device workspace that plx_decode needs for the
+ * given shape on the CURRENT device (it depends on the device's SM count).
+ * Returns 0 for an invalid shape.
+ */
+PLX_API size_t plx_decode_workspace_bytes(int B, int H_q, int H_kv, int d, int S_max);
+
+/*
+ * plx_decode -- single-token Parallax decode over a KV cache (page 3: a KV
+ * cache is still required for decoding).
+ *
+ *   q, rho           : [B, H_q, d]          the new token's queries and probes
+ *   k_cache, v_cache : [B, S_max, H_kv, d]  cached keys and values
+ *   seqlens          : [B] int32, device    batch b attends to cache rows
+ *                      0 .. seqlens[b]-1; values are clamped to [0, S_max];
+ *                      a length of 0 writes out = 0 for that batch
+ *   out              : [B, H_q, d]          written
+ *   workspace        : device memory of at least
+ *                      plx_decode_workspace_bytes(...) bytes, 16-byte aligned,
+ *                      contents need no initialisation; it must not be used
+ *                      by another call that may run concurrently.
+ * Rows beyond seqlens[b] (up to S_max) are never used, whatever they hold.
+ */
+PLX_API plx_status plx_decode(const void* q, const void* rho, const void* k_cache,
+                      const void* v_cache, const int32_t* seqlens, void* out, int B, int H_q,
+                      int H_kv, int d, int S_max, plx_dtype dtype, float softmax_scale,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+PLX_API const char* plx_status_string(plx_status s);
+
+/* cudaError_t behind this thread's last PLX_ERR_CUDA (0 if none). */
+PLX_API int plx_last_cuda_error(void);
+
+/*
+ * plx_device_error -- reads (and, if clear != 0, resets) the device-side error
+ * word of the current device: 0 = none, 1 = a bounded wait ran out of time,
+ * 2 = a kernel saw inconsistent internal state.  Synchronises the device.
+ * Returns PLX_OK or PLX_ERR_CUDA.
+ */
+PLX_API plx_status plx_device_error(int* code, int clear);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+PLX_API int plx_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PLX_H_ */

@@ -1,0 +1,106 @@
+"""The C ABI library: it loads, exports what include/plx.h declares, and its
+host-side argument checks reject bad calls before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from covariance_corrected_softmax_b200 import plx
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "plx.h")
+
+FAKE = 0x10000  # never dereferenced: every case below fails validation first
+
+
+def declared_symbols():
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"PLX_API\s+[\w\s\*]+?\b(plx_\w+)\s*\(", text)
+
+
+def test_header_declares_entry_points():
+    names = declared_symbols()
+    for n in ("plx_prefill_fwd", "plx_decode", "plx_decode_workspace_bytes",
+              "plx_status_string", "plx_last_cuda_error", "plx_device_error", "plx_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(plx.LIB_PATH)
+    for n in declared_symbols():
+        assert hasattr(lib, n), f"{n} declared in plx.h but not exported"
+
+
+def test_status_strings():
+    assert plx.status_string(0) == "PLX_OK"
+    assert plx.status_string(3) == "PLX_ERR_WORKSPACE_TOO_SMALL"
+    assert plx.lib().plx_version() >= 100
+
+
+def _decode(**kw):
+    a = dict(q=FAKE, rho=FAKE, k=FAKE, v=FAKE, sl=FAKE, out=FAKE, B=2, Hq=4, Hkv=2, d=128,
+             S=64, dtype=plx.PLX_BF16, scale=1.0, ws=FAKE, wsb=1 << 20)
+    a.update(kw)
+    return plx.lib().plx_decode(a["q"], a["rho"], a["k"], a["v"], a["sl"], a["out"], a["B"],
+                                a["Hq"], a["Hkv"], a["d"], a["S"], a["dtype"], a["scale"],
+                                a["ws"], a["wsb"], None)
+
+
+def _prefill(**kw):
+    a = dict(q=FAKE, rho=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=None, causal=1, B=1, L=16, Hq=2,
+             Hkv=1, d=64, dtype=plx.PLX_F32, scale=0.125)
+    a.update(kw)
+    return plx.lib().plx_prefill_fwd(a["q"], a["rho"], a["k"], a["v"], a["out"], a["lse"],
+                                     a["causal"], a["B"], a["L"], a["Hq"], a["Hkv"], a["d"],
+                                     a["dtype"], a["scale"], None)
+
+
+INV = plx.PLX_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("kw", [
+    dict(d=96), dict(d=0), dict(Hq=3, Hkv=2), dict(Hq=0), dict(Hkv=0), dict(B=-1), dict(S=0),
+    dict(dtype=7), dict(scale=float("nan")), dict(scale=float("inf")), dict(q=None),
+    dict(k=None), dict(sl=None), dict(ws=None), dict(out=None), dict(q=FAKE + 8),
+    dict(v=FAKE + 4), dict(ws=FAKE + 8), dict(sl=FAKE + 2),
+])
+def test_decode_rejects(kw):
+    assert _decode(**kw) == INV
+
+
+def test_decode_empty_batch_is_noop():
+    assert _decode(B=0, q=None, k=None) == plx.PLX_OK
+
+
+@pytest.mark.parametrize("kw", [
+    dict(d=32), dict(Hq=2, Hkv=3), dict(causal=2), dict(L=-1), dict(dtype=3),
+    dict(scale=float("nan")), dict(q=None), dict(rho=None), dict(out=None), dict(k=FAKE + 8),
+    dict(lse=FAKE + 2),
+])
+def test_prefill_rejects(kw):
+    assert _prefill(**kw) == INV
+
+
+def test_prefill_empty_is_noop():
+    assert _prefill(B=0, q=None) == plx.PLX_OK
+    assert _prefill(L=0, q=None) == plx.PLX_OK
+
+
+def test_workspace_query_rejects_bad_shapes():
+    L = plx.lib()
+    assert L.plx_decode_workspace_bytes(1, 3, 2, 128, 64) == 0
+    assert L.plx_decode_workspace_bytes(1, 2, 2, 80, 64) == 0
+    assert L.plx_decode_workspace_bytes(1, 2, 2, 64, 0) == 0
+
+
+def test_product_path_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "covariance_corrected_softmax_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                with open(os.path.join(dirpath, fn)) as f:
+                    src = f.read()
+                assert "import oracle" not in src and "from oracle" not in src, fn
+                assert "plx_oracle" not in src and "plxo_" not in src, fn
