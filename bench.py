@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Benchmark of the Parallax hot path on B200 (one JSON line on rank 0).
+
+Headline workload: single-token decode over a bf16 KV cache, B=32, H_q=16,
+H_kv=8, d=128, context 4096 (``decode_b32_ctx4096``).  One step is one
+``plx_decode`` call (score, probe score, online softmax, both accumulators,
+split merge).  The causal prefill rows of the hot path are measured in the same
+run on ``prefill_b8_l4096`` (B=8, L=4096, H_q=16, H_kv=8, d=128) and reported
+under ``"prefill"``.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
+a device synchronisation, timed with CUDA events on the launching stream; the
+elapsed time is the maximum over ranks.  The KV cache rotates over three
+independent copies of 537 MB each (inputs larger than the 126 MB L2), so every
+step reads its cache from HBM.
+
+Multi-GPU (torchrun, one process per GPU): the decode batches are independent
+problems, so every rank runs its own batch with no data-path collective
+("scaling": "weak"); value = all ranks' tokens / max-over-ranks time.
+
+``--impl reference`` times the fp64 CPU oracle instead (on rank 0 only), on the
+same workload and metric, one bounded sample of decode rows per step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s & HBM GB/s (% of roofline); prefill TFLOP/s (% bf16 peak)"
+HEADLINE = "decode_b32_ctx4096"
+PREFILL = "prefill_b8_l4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DECODE_SOURCES = ["plx_decode.cu", "plx_decode.cuh", "plx_device.cuh"]
+PREFILL_SOURCES = ["plx_prefill_tc.cu", "plx_device.cuh"]
+
+
+# --------------------------------------------------------------------------- util
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "covariance_corrected_softmax_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(kernel, workload, names):
+    """DRAM bytes per launch from profiles/dram_traffic.txt, if taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = source_digest(names)
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and \
+                    parts[1] == workload and parts[3] == digest:
+                return float(parts[2])
+    return None
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while it runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.idx = gpu_index
+        self.period = period_ms
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", str(self.period)],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            with open(self.path) as f:
+                for line in f:
+                    p = [x.strip() for x in line.split(",")]
+                    if len(p) < 9:
+                        continue
+                    try:
+                        rows.append((float(p[1]), float(p[2]), float(p[3]), p[5:9]))
+                    except ValueError:
+                        continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------ decode
+def decode_alg_bytes(shape, seqlens) -> float:
+    esz = 2
+    kv = float(seqlens.sum().item()) * shape.Hkv * shape.d * esz * 2
+    return kv + shape.B * shape.Hq * shape.d * esz * 3
+
+
+def bench_decode(plx, W, shape, steps, warmup, world, device, rank):
+    import torch
+    inp = W.make_decode(shape, seed=rank, device=device, copies=3)
+    ws = plx.decode_workspace(shape.B, shape.Hq, shape.Hkv, shape.d, shape.S_max, device=device)
+    out = torch.empty_like(inp["q"])
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        plx.decode(inp["q"], inp["rho"], inp["k_caches"][i % 3], inp["v_caches"][i % 3],
+                   inp["seqlens"], softmax_scale=1.0, out=out, workspace=ws, stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    gpu_idx = torch.cuda.current_device()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            gpu_idx = int(vis.split(",")[gpu_idx])
+        except (ValueError, IndexError):
+            pass
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_idx) as clk:
+        s.record(stream)
+        for i in range(steps):
+            step(warmup + i)
+        e.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    local_ms = s.elapsed_time(e)
+    total_ms = max_over_ranks(local_ms, world, device)
+    assert plx.device_error() == 0, "decode kernels reported a device error"
+    return {"ms": total_ms, "alg_bytes": decode_alg_bytes(shape, inp["seqlens"]),
+            "clocks": clk.summary(), "inp": inp}
+
+
+def bench_decode_e2e(plx, W, shape, steps, warmup, world, device, rank):
+    """Same metric through the public call with host I/O every step: the new
+    token's q, rho, k, v and the lengths go host -> device from pinned memory
+    (k, v written into the cache at the last position), and out comes back."""
+    import torch
+    inp = W.make_decode(shape, seed=100 + rank, device=device, copies=3)
+    B, Hq, Hkv, d = shape.B, shape.Hq, shape.Hkv, shape.d
+    pos = shape.ctx - 1
+    h = {
+        "q": inp["q"].cpu().pin_memory(),
+        "rho": inp["rho"].cpu().pin_memory(),
+        "k": inp["k_cache"][:, pos].contiguous().cpu().pin_memory(),
+        "v": inp["v_cache"][:, pos].contiguous().cpu().pin_memory(),
+        "sl": inp["seqlens"].cpu().pin_memory(),
+    }
+    out_h = torch.empty((B, Hq, d), dtype=inp["q"].dtype).pin_memory()
+    q_d, rho_d, sl_d = torch.empty_like(inp["q"]), torch.empty_like(inp["rho"]), \
+        torch.empty_like(inp["seqlens"])
+    out_d = torch.empty_like(inp["q"])
+    ws = plx.decode_workspace(B, Hq, Hkv, d, shape.S_max, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        kc, vc = inp["k_caches"][i % 3], inp["v_caches"][i % 3]
+        q_d.copy_(h["q"], non_blocking=True)
+        rho_d.copy_(h["rho"], non_blocking=True)
+        kc[:, pos].copy_(h["k"], non_blocking=True)
+        vc[:, pos].copy_(h["v"], non_blocking=True)
+        sl_d.copy_(h["sl"], non_blocking=True)
+        plx.decode(q_d, rho_d, kc, vc, sl_d, softmax_scale=1.0, out=out_d, workspace=ws,
+                   stream=stream)
+        out_h.copy_(out_d, non_blocking=True)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for i in range(steps):
+        step(warmup + i)
+    e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world, device)
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = out_h.numel() * out_h.element_size()
+    return {"ms": ms, "h2d": h2d, "d2h": d2h}
+
+
+def cpu_baseline_decode(inp, shape, seconds: float = 12.0):
+    """The oracle (explicit covariance form) on sampled rows of the same decode
+    batch, on all host cores; tokens/s = rows/s / H_q."""
+    import numpy as np
+    import oracle
+    from covariance_corrected_softmax_b200 import workloads as W
+    threads = oracle.default_threads()
+    q, rho = inp["q"].float().cpu(), inp["rho"].float().cpu()
+    kc, vc = inp["k_cache"], inp["v_cache"]
+    sl = inp["seqlens"].cpu()
+    rows = W.sample_rows_decode(shape.B, shape.Hq, shape.B * shape.Hq, seed=2)
+    done, t_used, n = 0, 0.0, max(1, threads)
+    while done < len(rows):
+        chunk = rows[done:done + n]
+        t0 = time.perf_counter()
+        oracle.decode(q, rho, kc, vc, sl, 1.0, rows=chunk, threads=threads)
+        t_used += time.perf_counter() - t0
+        done += len(chunk)
+        if t_used >= seconds:
+            break
+        n = min(4 * n, len(rows) - done) if t_used < seconds / 4 else n
+    rows_per_s = done / t_used
+    return {"value": rows_per_s / shape.Hq, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{done} of {shape.B * shape.Hq} (b, h) rows of {HEADLINE} "
+                      f"(explicit fp64 covariance form), {t_used:.1f} s"}
+
+
+# ----------------------------------------------------------------------- prefill
+def bench_prefill(plx, W, shape, steps, warmup, world, device, rank):
+    import torch
+    inp = [W.make_prefill(shape, seed=10 + rank + 7 * c, device=device) for c in range(2)]
+    out = torch.empty_like(inp[0]["q"])
+    lse = torch.empty((shape.B, shape.Hq, shape.L), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        x = inp[i % 2]
+        plx.prefill(x["q"], x["rho"], x["k"], x["v"], causal=shape.causal, softmax_scale=1.0,
+                    out=out, lse=lse, stream=stream)
+
+    try:
+        step(0)
+    except plx.PlxError as e:
+        return {"status": str(e)}
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for i in range(steps):
+        step(i)
+    e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world, device)
+    assert plx.device_error() == 0, "prefill kernel reported a device error"
+    return {"ms": ms}
+
+
+# -------------------------------------------------------------------- reference
+def reference_arm(args):
+    """The oracle as it stands on the host cores, same workload and metric."""
+    rank, _, world = env_rank()
+    if rank != 0:
+        return 0
+    import torch
+    import oracle
+    from covariance_corrected_softmax_b200 import workloads as W
+    shape = W.WORKLOADS[HEADLINE]
+    inp = W.make_decode(shape, seed=0, device="cpu")
+    threads = oracle.default_threads()
+    rows = W.sample_rows_decode(shape.B, shape.Hq, shape.B * shape.Hq, seed=3)
+    q, rho = inp["q"].float(), inp["rho"].float()
+    # A step is one row per host thread, evaluated in parallel; if K + W such
+    # steps would run past ~2.5 minutes, a step is a single row on one thread.
+    per_step = threads
+    t0 = time.perf_counter()
+    oracle.decode(q, rho, inp["k_cache"], inp["v_cache"], inp["seqlens"], 1.0,
+                  rows=rows[:per_step], threads=threads)
+    step_s = time.perf_counter() - t0
+    if (args.steps + args.warmup) * step_s > 150:
+        per_step = 1
+    used = min(threads, per_step)
+    k = 0
+
+    def run_step():
+        nonlocal k
+        idx = [(k + j) % len(rows) for j in range(per_step)]
+        k += per_step
+        oracle.decode(q, rho, inp["k_cache"], inp["v_cache"], inp["seqlens"], 1.0,
+                      rows=rows[idx], threads=used)
+
+    for _ in range(args.warmup):
+        run_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run_step()
+    secs = time.perf_counter() - t0
+    tok_s = args.steps * per_step / shape.Hq / secs
+    rec = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs * 1e3 / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": headline_config(shape, world),
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                         "sample": f"{per_step} (b, h) rows of {HEADLINE} per step "
+                                   "(explicit fp64 covariance form)"},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(rec), flush=True)
+    return 0
+
+
+def headline_config(shape, world):
+    return {"workload": HEADLINE, "B": shape.B, "H_q": shape.Hq, "H_kv": shape.Hkv,
+            "d": shape.d, "context": shape.ctx, "softmax_scale": 1.0,
+            "kv_cache_bytes": shape.B * shape.S_max * shape.Hkv * shape.d * 2 * 2,
+            "l2": "inputs larger than L2: 3 rotating KV cache copies of 537 MB",
+            "parallelism": f"replicas x{world} (independent decode batches per GPU)"}
+
+
+# ------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["plx", "reference"], default="plx")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-I/O leg (profiling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    from covariance_corrected_softmax_b200 import plx, workloads as W
+
+    rank, local_rank, world = env_rank()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    peaks, peak_src = load_peaks()
+
+    shape = W.WORKLOADS[HEADLINE]
+    dec = bench_decode(plx, W, shape, args.steps, args.warmup, world, device, rank)
+    ms_step = dec["ms"] / args.steps
+    tok_s = world * shape.B * args.steps / (dec["ms"] / 1e3)
+    gbs = dec["alg_bytes"] / (ms_step / 1e3) / 1e9
+    e2e_rec = None
+    if not args.no_e2e:
+        e2e = bench_decode_e2e(plx, W, shape, args.steps, args.warmup, world, device, rank)
+        e2e_rec = {"value": world * shape.B * args.steps / (e2e["ms"] / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                   "ms_per_step": e2e["ms"] / args.steps}
+
+    prefill = None
+    if not args.no_prefill:
+        pshape = W.WORKLOADS[PREFILL]
+        psteps = max(3, min(200, args.steps // 10))
+        pr = bench_prefill(plx, W, pshape, psteps, max(3, min(args.warmup, 10)), world, device,
+                           rank)
+        if "ms" in pr:
+            pms = pr["ms"] / psteps
+            tflops = pshape.flops() / (pms / 1e3) / 1e12
+            prefill = {
+                "workload": PREFILL, "B": pshape.B, "L": pshape.L, "H_q": pshape.Hq,
+                "H_kv": pshape.Hkv, "d": pshape.d, "causal": pshape.causal, "steps": psteps,
+                "ms_per_call": pms, "tflops": tflops,
+                "tokens_per_s": world * pshape.B * pshape.L / (pms / 1e3),
+                "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                             "peak_source": f"{peak_src} bf16 dense (burst)",
+                             "flops_per_call": pshape.flops(),
+                             "traffic": recorded_traffic("plx_prefill_tc", PREFILL,
+                                                         PREFILL_SOURCES)},
+                "gpu_launches_per_call": 1,
+            }
+        else:
+            prefill = {"workload": PREFILL, **pr}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_decode(dec["inp"], shape)
+
+    traffic = recorded_traffic("plx_decode", HEADLINE, DECODE_SOURCES)
+    rec = {
+        "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": headline_config(shape, world),
+        "hbm_gbs": gbs,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"],
+                     "kernel": "plx_decode (split-K main kernel + combine kernel)",
+                     "peak_source": f"{peak_src} HBM copy bandwidth",
+                     "bytes_per_call": dec["alg_bytes"], "traffic": traffic},
+        "cpu_baseline": cpu,
+        "e2e": e2e_rec,
+        "gpu_launches": 2 * args.steps,
+        "clocks": dec["clocks"],
+        "prefill": prefill,
+    }
+    if rank == 0:
+        print(json.dumps(rec), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
