@@ -99,6 +99,7 @@ bool shape_ok(int H_q, int H_kv, int d) {
 
 namespace plx {
 EncodeTiledFn tensor_map_encoder() { return get_encoder() == cudaSuccess ? g_encode : nullptr; }
+void set_last_cuda_error(int e) { t_last_cuda_error = e; }
 }  // namespace plx
 
 extern "C" {

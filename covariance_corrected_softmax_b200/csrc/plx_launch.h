@@ -49,4 +49,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn tensor_map_encoder();
 
+// Records a cudaError_t as this thread's plx_last_cuda_error().
+void set_last_cuda_error(int e);
+
 }  // namespace plx

@@ -116,6 +116,33 @@ PLX_API plx_status plx_decode(const void* q, const void* rho, const void* k_cach
                       int H_kv, int d, int S_max, plx_dtype dtype, float softmax_scale,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * plx_decode_static_ws -- plx_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this entry point: it is a service
+ * of the library.  Callers it serves: a serving loop that must not enter the
+ * device allocator on its per-token path (cudaMalloc can synchronise the
+ * device and stall), a plugin whose host framework owns the whole device
+ * memory pool, or a C caller with no device allocator at hand.
+ *
+ * Arguments and results are those of plx_decode without the workspace: the
+ * caller still passes every input and the output.  The workspace is a fixed
+ * 1 MiB array in the library's device memory, present on every GPU that loads
+ * the library until the process exits.  A shape whose workspace would exceed
+ * 1 MiB returns PLX_ERR_WORKSPACE_TOO_SMALL (B200's 148 SMs need about 0.6 MiB
+ * for d = 128, so every valid shape fits there).  No allocation of any kind.
+ *
+ * The first call on a device looks up the array's device address with
+ * cudaGetSymbolAddress (once per device, with that device current); make that
+ * first call before any stream capture.  Every call on a device shares the one
+ * array, so calls whose work may overlap on the GPU (different streams, host
+ * threads) race on it and must be serialised by the caller.  Its contents
+ * carry over between calls; nothing in it needs clearing.
+ */
+PLX_API plx_status plx_decode_static_ws(const void* q, const void* rho, const void* k_cache,
+                                        const void* v_cache, const int32_t* seqlens, void* out,
+                                        int B, int H_q, int H_kv, int d, int S_max,
+                                        plx_dtype dtype, float softmax_scale, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 PLX_API const char* plx_status_string(plx_status s);
 
