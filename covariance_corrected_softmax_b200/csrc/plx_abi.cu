@@ -200,9 +200,12 @@ plx_status plx_decode(const void* q, const void* rho, const void* k_cache, const
 
 plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k, const void* v,
                            void* out, float* lse, int causal, int B, int L, int H_q, int H_kv,
-                           int d, plx_dtype dtype, float softmax_scale, void* stream) {
+                           int d, plx_dtype dtype, plx_dtype out_dtype, float softmax_scale,
+                           void* stream) {
   t_last_cuda_error = 0;
   if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
+  if (out_dtype != dtype && !(dtype == PLX_BF16 && out_dtype == PLX_F32))
+    return PLX_ERR_INVALID_ARGUMENT;
   if (B < 0 || L < 0 || !shape_ok(H_q, H_kv, d) || (causal != 0 && causal != 1))
     return PLX_ERR_INVALID_ARGUMENT;
   if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
@@ -250,6 +253,7 @@ plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k, const 
   a.Hkv = H_kv;
   a.d = d;
   a.causal = causal;
+  a.out_f32 = out_dtype == PLX_F32 ? 1 : 0;
   a.scale = softmax_scale;
   a.err = err;
   a.num_sms = sms;

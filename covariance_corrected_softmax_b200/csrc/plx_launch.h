@@ -29,6 +29,7 @@ struct PrefillTcArgs {
   void* out;
   float* lse;
   int B, L, Hq, Hkv, d, causal;
+  int out_f32;  // 1: out is fp32, 0: out is bf16
   float scale;
   unsigned* err;
   int num_sms;

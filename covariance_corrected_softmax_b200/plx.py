@@ -44,7 +44,7 @@ def lib() -> ctypes.CDLL:
                 "`python -m covariance_corrected_softmax_b200.build` (or __graft_entry__.build())")
         L = ctypes.CDLL(LIB_PATH)
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-        L.plx_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp]
+        L.plx_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp]
         L.plx_prefill_fwd.restype = i
         L.plx_decode_workspace_bytes.argtypes = [i, i, i, i, i]
         L.plx_decode_workspace_bytes.restype = sz
@@ -98,12 +98,14 @@ def _same(ref: torch.Tensor, *ts: torch.Tensor) -> None:
 def prefill(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             causal: bool = True, softmax_scale: Optional[float] = None,
             return_lse: bool = True, out: Optional[torch.Tensor] = None,
-            lse: Optional[torch.Tensor] = None, stream=None
+            lse: Optional[torch.Tensor] = None, stream=None,
+            out_dtype: Optional[torch.dtype] = None
             ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Parallax attention forward: q, rho [B, L, Hq, d]; k, v [B, L, Hkv, d].
 
     Returns (out [B, L, Hq, d], lse [B, Hq, L] fp32 or None).  softmax_scale
-    defaults to 1/sqrt(d).
+    defaults to 1/sqrt(d); out_dtype defaults to the input dtype (torch.float32
+    is also accepted for bf16 inputs).
     """
     _same(q, rho, k, v)
     B, L, Hq, d = q.shape
@@ -112,12 +114,12 @@ def prefill(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch.Tensor
         raise ValueError("shape mismatch among q, rho, k, v")
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
     st = lib().plx_prefill_fwd(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out),
                                _ptr(lse) if return_lse else None, int(bool(causal)), B, L, Hq,
-                               Hkv, d, _dtype_code(q), scale, _stream(stream))
+                               Hkv, d, _dtype_code(q), _dtype_code(out), scale, _stream(stream))
     _check(st, "plx_prefill_fwd")
     return out, (lse if return_lse else None)
 

@@ -73,20 +73,27 @@ typedef enum plx_dtype { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
  *
  *   q, rho : [B, L, H_q, d]   queries and probes (one probe per query row)
  *   k, v   : [B, L, H_kv, d]  keys and values
- *   out    : [B, L, H_q, d]   written
+ *   out    : [B, L, H_q, d]   written, in out_dtype
  *   lse    : [B, H_q, L] fp32, written if non-NULL: natural-log
  *            log-sum-exp of the scaled scores of each row (the softmax
  *            normaliser; independent of rho)
  *   causal : 1 = row i sees keys 0..i; 0 = every row sees all L keys
+ *   dtype  : of q, rho, k, v
+ *   out_dtype : of out; equal to dtype, or PLX_F32 with bf16 inputs (an fp32
+ *            result avoids the final rounding to bf16's 8 significant bits)
  *   softmax_scale : the score scale (1/sqrt(d) in the textbook form,
  *            page 1 section 1.1); any finite value
  * Sizes: B, L, H_q, H_kv >= 1 (B == 0 or L == 0 is a no-op returning PLX_OK).
+ * PLX_BF16 computes S = q.k and t = rho.k from the bf16 inputs on the tensor
+ * cores and the two value products in fp16 x fp16 (fp32 accumulation), so
+ * |v| and |rho . k| must stay below 65504; a non-finite result sets device
+ * error 3 (plx_device_error).
  * Operator definition: page 1 section 1.3 and page 3 (see the file header).
  */
-PLX_API plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k, const void* v,
-                           void* out, float* lse, int causal, int B, int L, int H_q,
-                           int H_kv, int d, plx_dtype dtype, float softmax_scale,
-                           void* stream);
+PLX_API plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k,
+                                   const void* v, void* out, float* lse, int causal, int B,
+                                   int L, int H_q, int H_kv, int d, plx_dtype dtype,
+                                   plx_dtype out_dtype, float softmax_scale, void* stream);
 
 /*
  * plx_decode_workspace_bytes -- device workspace that plx_decode needs for the
@@ -152,7 +159,8 @@ PLX_API int plx_last_cuda_error(void);
 /*
  * plx_device_error -- reads (and, if clear != 0, resets) the device-side error
  * word of the current device: 0 = none, 1 = a bounded wait ran out of time,
- * 2 = a kernel saw inconsistent internal state.  Synchronises the device.
+ * 2 = a kernel saw inconsistent internal state, 3 = a result was not finite
+ * (inputs outside the supported range).  Synchronises the device.
  * Returns PLX_OK or PLX_ERR_CUDA.
  */
 PLX_API plx_status plx_device_error(int* code, int clear);

@@ -39,11 +39,14 @@ def check_out(gpu, ref, bf16: bool, what: str = "", output_rounding: bool = Fals
     err = np.max(np.abs(gpu - ref)) if gpu.size else 0.0
     if bf16:
         rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 1.0
+        diff = np.abs(gpu - ref)
         if output_rounding and gpu.size:
-            err = float(np.max(np.abs(gpu - ref) - 2.0 ** -8 * np.abs(ref)))
-            err = max(err, 0.0)
+            diff = np.maximum(diff - 2.0 ** -8 * np.abs(ref), 0.0)
+        err = float(diff.max()) if gpu.size else 0.0
         rel = err / max(rms, 1e-30)
-        assert rel <= BF16_REL_RMS, f"{what}: max err {err:.3e} / rms {rms:.3e} = {rel:.3e}"
+        where = np.unravel_index(int(np.argmax(diff)), diff.shape) if gpu.size else ()
+        assert rel <= BF16_REL_RMS, (f"{what}: max err {err:.3e} / rms {rms:.3e} = {rel:.3e} "
+                                     f"at {where} (gpu {gpu[where]:.5f}, ref {ref[where]:.5f})")
         return rel
     assert err <= FP32_ATOL, f"{what}: max abs err {err:.3e} > {FP32_ATOL}"
     return err

@@ -50,11 +50,12 @@ def _decode(**kw):
 
 def _prefill(**kw):
     a = dict(q=FAKE, rho=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=None, causal=1, B=1, L=16, Hq=2,
-             Hkv=1, d=64, dtype=plx.PLX_F32, scale=0.125)
+             Hkv=1, d=64, dtype=plx.PLX_F32, out_dtype=None, scale=0.125)
     a.update(kw)
+    od = a["dtype"] if a["out_dtype"] is None else a["out_dtype"]
     return plx.lib().plx_prefill_fwd(a["q"], a["rho"], a["k"], a["v"], a["out"], a["lse"],
                                      a["causal"], a["B"], a["L"], a["Hq"], a["Hkv"], a["d"],
-                                     a["dtype"], a["scale"], None)
+                                     a["dtype"], od, a["scale"], None)
 
 
 INV = plx.PLX_ERR_INVALID_ARGUMENT
@@ -77,7 +78,7 @@ def test_decode_empty_batch_is_noop():
 @pytest.mark.parametrize("kw", [
     dict(d=32), dict(Hq=2, Hkv=3), dict(causal=2), dict(L=-1), dict(dtype=3),
     dict(scale=float("nan")), dict(q=None), dict(rho=None), dict(out=None), dict(k=FAKE + 8),
-    dict(lse=FAKE + 2),
+    dict(lse=FAKE + 2), dict(out_dtype=plx.PLX_BF16), dict(out_dtype=5),
 ])
 def test_prefill_rejects(kw):
     assert _prefill(**kw) == INV
