@@ -17,7 +17,10 @@
 //   warp 1      MMA issuer (one thread): S = Q K^T and T = R K^T share the K
 //               tile; O += P V and U += (P o T) V share the V tile.
 //   warp 2      allocates / frees the 512 TMEM columns.
-//   warps 4-7   softmax + epilogue, one thread per query row (= TMEM lane).
+//   warps 4-11  softmax + epilogue: two warpgroups; thread (row, half) owns
+//               one query row (= TMEM lane) and half of each key tile's
+//               columns.  The partners of a row exchange their partial row
+//               maxima through shared memory once per tile.
 // TMEM columns: O [0, d), U [d, 2d), S buffers at 256 + 64 b, T buffers at
 // 384 + 64 b (b = tile parity): the tensor core computes S, T of tile j+1 while
 // the softmax warps turn S, T of tile j into P = 2^(s - m) and P t, which
@@ -41,8 +44,10 @@ namespace {
 
 constexpr int kBM = 128;      // query rows per tile = TMEM lanes
 constexpr int kBN = 64;       // keys per tile
+constexpr int kHalf = kBN / 2;  // key columns per softmax thread
 constexpr int kStages = 4;    // K/V ring depth
-constexpr int kThreads = 256;
+constexpr int kSoftWarps = 8;   // two softmax warpgroups
+constexpr int kThreads = (4 + kSoftWarps) * 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
@@ -60,6 +65,12 @@ struct TcCfg {
   static constexpr uint32_t IDESC_ST = umma_idesc_f16kind(kBM, kBN, false, false);
   static constexpr uint32_t IDESC_PV = umma_idesc_f16kind(kBM, D, true, true);
 };
+
+// Within an S (or T) buffer of 64 fp32 columns, the softmax half h writes its
+// 32 keys' fp16 values (16 packed columns) over the start of its own 32-column
+// range, so no half overwrites columns its partner has not read yet.  The PV
+// product's K-step kk (keys 16 kk .. 16 kk + 15) reads 8 packed columns at:
+__host__ __device__ constexpr uint32_t p_col(int kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
 
 struct TcParams {
   int B, L, Hq, Hkv, G, causal, nqt, units;
@@ -91,6 +102,13 @@ struct Bars {
   uint64_t s_full[2], p_full[2], o_done[2];
 };
 
+// Shared memory the two halves of a row exchange through (two slots, used
+// alternately, so one named barrier per exchange suffices).
+struct Xchg {
+  float2 tile[2][2][kBM];   // [slot][half][row]: (partial max, partial max |t|)
+  float4 sums[2][kBM];      // [half][row]: (l, z, l32, -)
+};
+
 template <int D, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     plx_prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap,
@@ -104,7 +122,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sR = smem + C::Q_BYTES;
   uint8_t* sKV = smem + 2 * C::Q_BYTES;
-  Bars* bars = reinterpret_cast<Bars*>(smem + C::TILE_SMEM);
+  Xchg* xch = reinterpret_cast<Xchg*>(smem + C::TILE_SMEM);
+  Bars* bars = reinterpret_cast<Bars*>(xch + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -121,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], kBM);
+      mbar_init(&bars->p_full[b], kSoftWarps);  // one arrival per softmax warp
       mbar_init(&bars->o_done[b], 1);
     }
     fence_mbarrier_init();
@@ -180,66 +199,100 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Issues, whichever is ready first, the S/T products of the next key tile
+    // (its K tile has landed and its TMEM buffer is free, i.e. the PV products
+    // of the tile two back have been issued) or the PV products of the oldest
+    // tile whose P has been written.  The tensor core runs them in issue order.
     if (lane == 0) {
-      const uint32_t sq = smem_u32(sQ), sr = smem_u32(sR), skv = smem_u32(sKV);
-      int g = 0, ku = 0;
-      bool ok = true;
-      auto issue_pv = [&](int t, bool first) -> bool {
-        const int b = t & 1, st = t % kStages;
-        if (!mbar_wait(&bars->p_full[b], (t >> 1) & 1, abort_flag, p.err)) return false;
-        tc_fence_after();
-        const uint32_t sv = skv + st * C::STAGE_BYTES + C::KV_BYTES;
+      // Descriptors are built once; a tile or k-step only moves the start
+      // address, i.e. adds (byte offset >> 4) to the low bits.
+      const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dr = smem_desc_sw128(smem_u32(sR), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t dv = smem_desc_sw128(smem_u32(sKV) + C::KV_BYTES, C::KV_BOX, 1024);
+      int total = 0;
+      for (int u = blockIdx.x; u < p.units; u += gridDim.x) total += unit_of(p, u).n;
+      int us = blockIdx.x, js = 0, kus = 0, ns = us < p.units ? unit_of(p, us).n : 0;
+      int up = blockIdx.x, jp = 0, np = ns;
+      int ts = 0, tp = 0;
+      bool qok = false;
+      uint64_t idle_since = globaltimer_ns();
+      uint32_t spins = 0;
+      while (tp < total) {
+        bool did = false;
+        if (ts < total && ts <= tp + 1) {
+          if (js == 0 && !qok) qok = mbar_test(&bars->q_full, kus & 1);
+          const int st = ts % kStages;
+          if ((js > 0 || qok) && mbar_test(&bars->kv_full[st], (ts / kStages) & 1)) {
+            tc_fence_after();
+            const int b = ts & 1;
+            const uint64_t bk0 = dk + (uint64_t)((st * C::STAGE_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bv = smem_desc_sw128(sv + kk * 16 * 128, C::KV_BOX, 1024);
-          umma_ts(tbase + C::COL_O, tbase + C::COL_S + 64 * b + kk * 8, bv, C::IDESC_PV,
-                  (first && kk == 0) ? 0u : 1u);
-        }
+            for (int k = 0; k < D / 16; ++k) {
+              const uint32_t off = ((k >> 2) * C::Q_BOX + (k & 3) * 32) >> 4;
+              const uint32_t koff = ((k >> 2) * C::KV_BOX + (k & 3) * 32) >> 4;
+              umma_ss(tbase + C::COL_S + 64 * b, dq + off, bk0 + koff, C::IDESC_ST,
+                      k > 0 ? 1u : 0u);
+            }
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bv = smem_desc_sw128(sv + kk * 16 * 128, C::KV_BOX, 1024);
-          umma_ts(tbase + C::COL_U, tbase + C::COL_T + 64 * b + kk * 8, bv, C::IDESC_PV,
-                  (first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(&bars->o_done[b]);
-        umma_commit(&bars->kv_empty[st]);
-        return true;
-      };
-      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ku) {
-        const Unit x = unit_of(p, u);
-        if (!mbar_wait(&bars->q_full, ku & 1, abort_flag, p.err)) break;
-        tc_fence_after();
-        for (int j = 0; j < x.n; ++j) {
-          const int t = g + j, st = t % kStages, b = t & 1;
-          if (!mbar_wait(&bars->kv_full[st], (t / kStages) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
+            for (int k = 0; k < D / 16; ++k) {
+              const uint32_t off = ((k >> 2) * C::Q_BOX + (k & 3) * 32) >> 4;
+              const uint32_t koff = ((k >> 2) * C::KV_BOX + (k & 3) * 32) >> 4;
+              umma_ss(tbase + C::COL_T + 64 * b, dr + off, bk0 + koff, C::IDESC_ST,
+                      k > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars->s_full[b]);
+            if (js == ns - 1) {
+              umma_commit(&bars->q_empty);  // Q and R of this unit are no longer read
+              us += gridDim.x;
+              ++kus;
+              js = 0;
+              qok = false;
+              ns = us < p.units ? unit_of(p, us).n : 0;
+            } else {
+              ++js;
+            }
+            ++ts;
+            did = true;
           }
+        }
+        if (!did && tp < ts && mbar_test(&bars->p_full[tp & 1], (tp >> 1) & 1)) {
           tc_fence_after();
-          const uint32_t sk = skv + st * C::STAGE_BYTES;
+          const int b = tp & 1, st = tp % kStages;
+          const uint64_t bv0 = dv + (uint64_t)((st * C::STAGE_BYTES) >> 4);
+          const bool first = jp == 0;
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * C::Q_BOX + (k & 3) * 32;
-            const uint32_t koff = (k >> 2) * C::KV_BOX + (k & 3) * 32;
-            umma_ss(tbase + C::COL_S + 64 * b, smem_desc_sw128(sq + off, 16, 1024),
-                    smem_desc_sw128(sk + koff, 16, 1024), C::IDESC_ST, k > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_ts(tbase + C::COL_O, tbase + C::COL_S + 64 * b + p_col(kk),
+                    bv0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+                    (first && kk == 0) ? 0u : 1u);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * C::Q_BOX + (k & 3) * 32;
-            const uint32_t koff = (k >> 2) * C::KV_BOX + (k & 3) * 32;
-            umma_ss(tbase + C::COL_T + 64 * b, smem_desc_sw128(sr + off, 16, 1024),
-                    smem_desc_sw128(sk + koff, 16, 1024), C::IDESC_ST, k > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_ts(tbase + C::COL_U, tbase + C::COL_T + 64 * b + p_col(kk),
+                    bv0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+                    (first && kk == 0) ? 0u : 1u);
+          umma_commit(&bars->o_done[b]);
+          umma_commit(&bars->kv_empty[st]);
+          if (jp == np - 1) {
+            up += gridDim.x;
+            jp = 0;
+            np = up < p.units ? unit_of(p, up).n : 0;
+          } else {
+            ++jp;
           }
-          umma_commit(&bars->s_full[b]);
-          if (j == x.n - 1) umma_commit(&bars->q_empty);
-          if (j > 0 && !issue_pv(t - 1, j == 1)) {
-            ok = false;
+          ++tp;
+          did = true;
+        }
+        if (did) {
+          idle_since = globaltimer_ns();
+        } else if ((++spins & 255u) == 0) {
+          if (*abort_flag) break;
+          if (globaltimer_ns() - idle_since > kWaitLimitNs) {
+            record_error(p.err, kDevTimeoutMbarrier);
+            *abort_flag = 1;
             break;
           }
         }
-        if (ok && !issue_pv(g + x.n - 1, x.n == 1)) ok = false;
-        g += x.n;
       }
       // Every MMA must have completed before the columns are released.
       umma_commit(&bars->drain);
@@ -249,18 +302,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
-    const int r = tid - 128;                       // row within the tile = TMEM lane
-    const uint32_t lane_addr = tbase + ((uint32_t)((warp - 4) * 32) << 16);
+    const int si = tid - 128;                      // 0 .. 255
+    const int half = si >> 7;                      // which 32 keys of each tile
+    const int qd = warp & 3;                       // TMEM lane quadrant
+    const int r = qd * 32 + lane;                  // row within the tile = TMEM lane
+    const uint32_t lane_addr = tbase + ((uint32_t)(qd * 32) << 16);
+    const uint32_t my_cols = (uint32_t)(half * kHalf);  // first S/T column of this half
+    const int bar_id = 1 + qd;                     // named barrier of the row's two warps
     const bool qpos = p.qscale >= 0.f;
-    int g = 0;
+    int g = 0, xs = 0;
     bool ok = true, finite = true;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
       const Unit x = unit_of(p, u);
       const int i = x.mt * kBM + r;
       // Running max m (log2 units of the scaled scores); P = 2^(s - m) <= 2^8
-      // (lazy rescaling).  l = sum P and z = sum P t * 2^-eu are summed from the
-      // rounded fp16 values the tensor core multiplies; l32 = sum P unrounded
-      // (for lse).  eu (>= 0) keeps P t * 2^-eu inside fp16's range.
+      // (lazy rescaling).  Per half: l = sum P and z = sum P t 2^-eu summed
+      // from the rounded fp16 values the tensor core multiplies, and l32 = sum
+      // P unrounded (for lse).  eu (>= 0) keeps P t 2^-eu inside fp16's range.
       float m_run = -INFINITY, l = 0.f, z = 0.f, l32 = 0.f;
       int eu = 0;
       for (int j = 0; j < x.n; ++j) {
@@ -273,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           uint4* vt = reinterpret_cast<uint4*>(sKV + st * C::STAGE_BYTES + C::KV_BYTES);
 #pragma unroll
-          for (int c = r; c < C::KV_BYTES / 16; c += kBM) {
+          for (int c = si; c < C::KV_BYTES / 16; c += kSoftWarps * 32) {
             uint4 w = vt[c];
             float2 f;
             f = bf16x2_to_float2(w.x);
@@ -293,33 +351,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sv[64], tv[64];
-        {
-          uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
-          uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-          tmem_ld2x32_sync(lane_addr + C::COL_S + 64 * b, lane_addr + C::COL_S + 64 * b + 32, s0,
-                           s1);
-          uint32_t (&t0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&tv[0]);
-          uint32_t (&t1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&tv[32]);
-          tmem_ld2x32_sync(lane_addr + C::COL_T + 64 * b, lane_addr + C::COL_T + 64 * b + 32, t0,
-                           t1);
-        }
-        const int key0 = j * kBN;
-        const bool need_mask = p.causal ? (key0 + kBN - 1 > i) : (key0 + kBN > p.L);
-        const int nvis = need_mask ? max(0, min(kBN, (p.causal ? i : p.L - 1) - key0 + 1)) : kBN;
-        // extreme of the raw scores (max if scale >= 0) and max |t| over the
-        // visible keys
-        float ext = qpos ? -INFINITY : INFINITY, tmax = 0.f;
+        uint32_t sv[kHalf], tv[kHalf];
+        tmem_ld2x32_sync(lane_addr + C::COL_S + 64 * b + my_cols,
+                         lane_addr + C::COL_T + 64 * b + my_cols, sv, tv);
+        const int key0 = j * kBN + half * kHalf;  // first key of this half
+        const int lim = p.causal ? i : p.L - 1;    // last visible key of the row
+        const int nvis = max(0, min(kHalf, lim - key0 + 1));
+        // partial extreme of the raw scores (max if scale >= 0) and max |t|
+        float e4[4], t4[4];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float v = __uint_as_float(sv[c]);
-          if (c < nvis) {
-            ext = qpos ? fmaxf(ext, v) : fminf(ext, v);
-            tmax = fmaxf(tmax, fabsf(__uint_as_float(tv[c])));
+        for (int q = 0; q < 4; ++q) {
+          e4[q] = qpos ? -INFINITY : INFINITY;
+          t4[q] = 0.f;
+        }
+        if (nvis == kHalf) {
+#pragma unroll
+          for (int c = 0; c < kHalf; ++c) {
+            const float v = __uint_as_float(sv[c]);
+            e4[c & 3] = qpos ? fmaxf(e4[c & 3], v) : fminf(e4[c & 3], v);
+            t4[c & 3] = fmaxf(t4[c & 3], fabsf(__uint_as_float(tv[c])));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kHalf; ++c) {
+            const float v = __uint_as_float(sv[c]);
+            if (c < nvis) {
+              e4[c & 3] = qpos ? fmaxf(e4[c & 3], v) : fminf(e4[c & 3], v);
+              t4[c & 3] = fmaxf(t4[c & 3], fabsf(__uint_as_float(tv[c])));
+            }
           }
         }
-        const float tile_max = (nvis > 0) ? ext * p.qscale : -INFINITY;
-        const float m_new = fmaxf(m_run, tile_max);
+        const float ext = qpos ? fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]))
+                               : fminf(fminf(e4[0], e4[1]), fminf(e4[2], e4[3]));
+        float part_max = (nvis > 0) ? ext * p.qscale : -INFINITY;
+        float tmax = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
+        // combine with the partner half of the row
+        xch->tile[xs & 1][half][r] = make_float2(part_max, tmax);
+        named_bar_sync(bar_id, 64);
+        {
+          const float2 o = xch->tile[xs & 1][half ^ 1][r];
+          part_max = fmaxf(part_max, o.x);
+          tmax = fmaxf(tmax, o.y);
+        }
+        ++xs;
+        const float m_new = fmaxf(m_run, part_max);
         const bool resc = (m_run != -INFINITY) && (m_new > m_run + kRescaleThreshold);
         if (m_run == -INFINITY) m_run = m_new;
         // |P t| <= 2^8 |t|: keep |t| 2^-eu below 2^7 (P t 2^-eu below 2^15)
@@ -327,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tmax * exp2f((float)-eu) >= 128.f) eu_new = max(eu, (int)ceilf(log2f(tmax)) - 6);
         const bool ubump = eu_new > eu;
         if (__any_sync(0xffffffffu, resc || ubump)) {
+          // (the partner warp holds the same rows and takes this branch too)
           if (j > 0 &&
               !mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag, p.err)) {
             ok = false;
@@ -335,14 +411,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const float alpha = resc ? exp2f(m_run - m_new) : 1.f;
           const float beta = alpha * exp2f((float)(eu - eu_new));
+          const float f = half == 0 ? alpha : beta;  // half 0 rescales O, half 1 rescales U
+          const uint32_t base = half == 0 ? C::COL_O : C::COL_U;
 #pragma unroll 1
-          for (int cc = 0; cc < 2 * D; cc += 32) {
-            const float f = cc < D ? alpha : beta;
+          for (int cc = 0; cc < D; cc += 32) {
             uint32_t w[32];
-            tmem_ld32_sync(lane_addr + C::COL_O + cc, w);
+            tmem_ld32_sync(lane_addr + base + cc, w);
 #pragma unroll
             for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
-            tmem_st32(lane_addr + C::COL_O + cc, w);
+            tmem_st32(lane_addr + base + cc, w);
           }
           tmem_wait_st();
           l *= alpha;
@@ -351,40 +428,63 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (resc) m_run = m_new;
           eu = eu_new;
         }
-        // P = 2^(s - m) as fp16 over the S buffer
+        // P = 2^(s - m) as fp16 over the start of this half's S columns
         const bool live = m_run != -INFINITY;
-        uint32_t pk[32];
+        uint32_t pk[kHalf / 2];
+        float2 la = make_float2(0.f, 0.f), lb = la, ra = la, rb = la;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          float p0 = exp2f(fmaf(__uint_as_float(sv[2 * c]), p.qscale, -m_run));
-          float p1 = exp2f(fmaf(__uint_as_float(sv[2 * c + 1]), p.qscale, -m_run));
+        for (int c = 0; c < kHalf / 2; ++c) {
+          float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), p.qscale, -m_run));
+          float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), p.qscale, -m_run));
           if (!live || 2 * c >= nvis) p0 = 0.f;
           if (!live || 2 * c + 1 >= nvis) p1 = 0.f;
           sv[2 * c] = __float_as_uint(p0);
           sv[2 * c + 1] = __float_as_uint(p1);
-          l32 += p0 + p1;
           pk[c] = float2_to_f16x2(p0, p1);
           const float2 rp = f16x2_to_float2(pk[c]);
-          l += rp.x + rp.y;
+          if (c & 1) {
+            lb = __fadd2_rn(lb, make_float2(p0, p1));
+            rb = __fadd2_rn(rb, rp);
+          } else {
+            la = __fadd2_rn(la, make_float2(p0, p1));
+            ra = __fadd2_rn(ra, rp);
+          }
         }
-        tmem_st32(lane_addr + C::COL_S + 64 * b, pk);
-        // P t 2^-eu as fp16 over the T buffer
+        l32 += (la.x + la.y) + (lb.x + lb.y);
+        l += (ra.x + ra.y) + (rb.x + rb.y);
+        tmem_st16(lane_addr + C::COL_S + 64 * b + my_cols, pk);
+        // P t 2^-eu as fp16 over the start of this half's T columns
         const float tsc = exp2f((float)-eu);
+        float2 za = make_float2(0.f, 0.f), zb = za;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < kHalf / 2; ++c) {
           const float q0 = __uint_as_float(sv[2 * c]) * (__uint_as_float(tv[2 * c]) * tsc);
           const float q1 = __uint_as_float(sv[2 * c + 1]) * (__uint_as_float(tv[2 * c + 1]) * tsc);
           pk[c] = float2_to_f16x2(q0, q1);
           const float2 rq = f16x2_to_float2(pk[c]);
-          z += rq.x + rq.y;
+          if (c & 1)
+            zb = __fadd2_rn(zb, rq);
+          else
+            za = __fadd2_rn(za, rq);
         }
-        tmem_st32(lane_addr + C::COL_T + 64 * b, pk);
+        z += (za.x + za.y) + (zb.x + zb.y);
+        tmem_st16(lane_addr + C::COL_T + 64 * b + my_cols, pk);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[b]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[b]);
       }
       if (!ok) break;
-      // ---- epilogue: out = ((1 + z/l) o - u) / l, lse = ln(sum exp(scale s))
+      // ---- epilogue: out = ((1 + z/l) o - u) / l, lse = ln(sum exp(scale s));
+      // the halves add their sums, then each writes half of the row.
+      xch->sums[half][r] = make_float4(l, z, l32, 0.f);
+      named_bar_sync(bar_id, 64);
+      {
+        const float4 o = xch->sums[half ^ 1][r];
+        l += o.x;
+        z += o.y;
+        l32 += o.z;
+      }
       const int tl = g + x.n - 1;
       if (!mbar_wait(&bars->o_done[tl & 1], (tl >> 1) & 1, abort_flag, p.err)) break;
       tc_fence_after();
@@ -394,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float cu = usc * inv;
       OutT* orow = static_cast<OutT*>(p.out) + (((size_t)x.b * p.L + i) * p.Hq + x.h) * D;
 #pragma unroll 1
-      for (int cc = 0; cc < D; cc += 32) {
+      for (int cc = half * (D / 2); cc < (half + 1) * (D / 2); cc += 32) {
         uint32_t ov[32], uv[32];
         tmem_ld2x32_sync(lane_addr + C::COL_O + cc, lane_addr + C::COL_U + cc, ov, uv);
         float a[32];
@@ -420,9 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (p.lse && i < p.L)
-        p.lse[((size_t)x.b * p.Hq + x.h) * p.L + i] =
-            (m_run + log2f(l32)) * 0.6931471805599453f;
+      if (half == 0 && p.lse && i < p.L)
+        p.lse[((size_t)x.b * p.Hq + x.h) * p.L + i] = (m_run + log2f(l32)) * 0.6931471805599453f;
       tc_fence_before();
       g += x.n;
     }
@@ -477,7 +576,7 @@ cudaError_t launch_d(const PrefillTcArgs& a, cudaStream_t stream) {
   p.out = a.out;
   p.lse = a.lse;
   p.err = a.err;
-  const int smem = 1024 + C::TILE_SMEM + (int)sizeof(Bars) + 16;
+  const int smem = 1024 + C::TILE_SMEM + (int)sizeof(Xchg) + (int)sizeof(Bars) + 16;
   auto kern = plx_prefill_tc_kernel<D, OutT>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
