@@ -159,7 +159,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   RangeInfo* info = reinterpret_cast<RangeInfo*>(empty + STAGES);
   long long* scan_ws = reinterpret_cast<long long*>(info + 1);   // 16 entries
   volatile int* abort_flag = reinterpret_cast<volatile int*>(scan_ws + 16);
-  float* merge = reinterpret_cast<float*>(scan_ws + 20);          // 16-byte aligned
+  float* merge = reinterpret_cast<float*>(scan_ws + 20);
+  float* red_smem = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(merge + kDecConsumerWarps * HPW * PHF) + 15) & ~uintptr_t(15));
+  float* bc_smem = red_smem + 2 * kDecConsumerWarps * kDecRedRegion;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -242,14 +245,25 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // ------------------------------------------------------------ consumers
     const int hw = lane >> 4, sub = lane & 15;
     const int rowbase = (warp * 2 + hw) * KPH;
+    // Per key, the half-warp forms 2 HPW partial dot products per lane (s for
+    // each head, then t for each head).  They are reduced by a transpose through
+    // shared memory: lane v ends up holding the full sum of value v, i.e. of
+    // kind v % NT for key v / NT of this half-warp's KPH keys.
+    constexpr int NT = 2 * HPW;
+    constexpr int NV = KPH * NT;
+    static_assert(NV <= 16 && (NV & (NV - 1)) == 0, "one reduced value per lane");
+    const int kv = sub / NT, kind = sub % NT;
+    const bool is_s = kind < HPW;              // a score lane (else a probe-score lane)
+    const int hsrc = lane - (is_s ? 0 : HPW);  // the score lane of the same key and head
+    const int hbase = lane & 16;               // first lane of this half-warp
+    float* red = red_smem + (warp * 2 + hw) * kDecRedRegion;
+    float* bc = bc_smem + (warp * 2 + hw) * 16;
     float2 qf[HPW][H2], rf[HPW][H2], oa[HPW][H2], ua[HPW][H2];
-    float m[HPW], l[HPW], z[HPW];
+    // running max of this lane's head, and l (score lanes) or z (probe lanes)
+    float m_run = -INFINITY, lz = 0.f;
     int ordinal = 0;
 #pragma unroll
     for (int g = 0; g < HPW; ++g) {
-      m[g] = -INFINITY;
-      l[g] = 0.f;
-      z[g] = 0.f;
 #pragma unroll
       for (int e = 0; e < H2; ++e) {
         qf[g][e] = rf[g][e] = oa[g][e] = ua[g][e] = make_float2(0.f, 0.f);
@@ -274,10 +288,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             qf[g][e].y *= p.qscale;
             oa[g][e] = ua[g][e] = make_float2(0.f, 0.f);
           }
-          m[g] = -INFINITY;
-          l[g] = 0.f;
-          z[g] = 0.f;
         }
+        m_run = -INFINITY;
+        lz = 0.f;
       }
 
       const uint8_t* kt_base = ring + stage * Cfg::STAGE_BYTES +
@@ -285,7 +298,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const uint8_t* vt_base = kt_base + Cfg::TILE_BYTES;
 
       // Phase A: partial dot products s = (scale log2e) q.k and t = rho.k
-      float s[KPH][HPW], tt[KPH][HPW];
+      float vals[NV];
 #pragma unroll
       for (int kk = 0; kk < KPH; ++kk) {
         float2 kf[H2];
@@ -298,62 +311,78 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             as = __ffma2_rn(qf[g][e], kf[e], as);
             at = __ffma2_rn(rf[g][e], kf[e], at);
           }
-          s[kk][g] = as.x + as.y;
-          tt[kk][g] = at.x + at.y;
+          vals[kk * NT + g] = as.x + as.y;
+          vals[kk * NT + HPW + g] = at.x + at.y;
         }
       }
-      // Phase B: reduce over the 16 lanes of the half-warp
+      // Phase B: transpose-reduce over the 16 lanes of the half-warp
 #pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) {
+      for (int q4 = 0; q4 < NV; q4 += 4)
+        *reinterpret_cast<float4*>(red + sub * kDecRedRow + q4) =
+            make_float4(vals[q4], vals[q4 + 1], vals[q4 + 2], vals[q4 + 3]);
+      __syncwarp();
+      float acc = 0.f;
+      if (sub < NV) {
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < KPH; ++kk) {
-#pragma unroll
-          for (int g = 0; g < HPW; ++g) {
-            s[kk][g] += __shfl_xor_sync(0xffffffffu, s[kk][g], off);
-            tt[kk][g] += __shfl_xor_sync(0xffffffffu, tt[kk][g], off);
-          }
+        for (int row = 0; row < 16; row += 2) {
+          a0 += red[row * kDecRedRow + sub];
+          a1 += red[(row + 1) * kDecRedRow + sub];
         }
+        acc = a0 + a1;
       }
-      // Phase C: online softmax over this half-warp's KPH keys
-      bool valid[KPH];
+      // Phase C: online softmax on the distributed values
+      const bool valid_k = (sub < NV) && (rowbase + kv) < mt.nvalid;
+      float val = acc;
+      if (is_s && !valid_k) val = -INFINITY;
+      float mx = val;
 #pragma unroll
-      for (int kk = 0; kk < KPH; ++kk) valid[kk] = (rowbase + kk) < mt.nvalid;
+      for (int o = NT; o < NV; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float smax = __shfl_sync(0xffffffffu, mx, hsrc);   // tile max of this head
+      float alpha = 1.f;
+      if (smax > m_run) {
+        alpha = merge_weight(m_run, smax);
+        lz *= alpha;
+        m_run = smax;
+      }
+      const float pv = is_s ? exp2_shift(val, m_run) : 0.f;
+      const float ps = __shfl_sync(0xffffffffu, pv, hsrc);
+      const float w = is_s ? pv : (valid_k ? ps * val : 0.f);  // p, or p t
+      float sw = w;
+#pragma unroll
+      for (int o = NT; o < NV; o <<= 1) sw += __shfl_xor_sync(0xffffffffu, sw, o);
+      lz += sw;
+      float al[HPW];
+#pragma unroll
+      for (int g = 0; g < HPW; ++g) al[g] = __shfl_sync(0xffffffffu, alpha, hbase + g);
+      if (sub < NV) bc[sub] = w;
+      __syncwarp();
       float pw[KPH][HPW], ptw[KPH][HPW];
 #pragma unroll
-      for (int g = 0; g < HPW; ++g) {
-        float mx = -INFINITY;
+      for (int kk = 0; kk < KPH; ++kk) {
 #pragma unroll
-        for (int kk = 0; kk < KPH; ++kk) {
-          if (!valid[kk]) s[kk][g] = -INFINITY;
-          mx = fmaxf(mx, s[kk][g]);
+        for (int g = 0; g < HPW; ++g) {
+          pw[kk][g] = bc[kk * NT + g];
+          ptw[kk][g] = bc[kk * NT + HPW + g];
         }
-        if (mx > m[g]) {
-          const float alpha = merge_weight(m[g], mx);
-          l[g] *= alpha;
-          z[g] *= alpha;
+      }
+#pragma unroll
+      for (int g = 0; g < HPW; ++g) {
+        if (al[g] != 1.f) {
 #pragma unroll
           for (int e = 0; e < H2; ++e) {
-            oa[g][e] = __fmul2_rn(oa[g][e], f2(alpha));
-            ua[g][e] = __fmul2_rn(ua[g][e], f2(alpha));
+            oa[g][e] = __fmul2_rn(oa[g][e], f2(al[g]));
+            ua[g][e] = __fmul2_rn(ua[g][e], f2(al[g]));
           }
-          m[g] = mx;
-        }
-#pragma unroll
-        for (int kk = 0; kk < KPH; ++kk) {
-          const float pr = exp2_shift(s[kk][g], m[g]);
-          const float pt = pr * tt[kk][g];
-          pw[kk][g] = pr;
-          ptw[kk][g] = valid[kk] ? pt : 0.f;
-          l[g] += pr;
-          z[g] += ptw[kk][g];
         }
       }
       // Phase D: accumulate o += p v and u += (p t) v
+      const bool tail = mt.nvalid < TK;
 #pragma unroll
       for (int kk = 0; kk < KPH; ++kk) {
         float2 vf[H2];
         RowLoad<T, EPL>::load(vt_base + kk * Cfg::ROW_BYTES, vf);
-        if (!valid[kk]) {
+        if (tail && rowbase + kk >= mt.nvalid) {  // rows past the length may hold anything
 #pragma unroll
           for (int e = 0; e < H2; ++e) vf[e] = make_float2(0.f, 0.f);
         }
@@ -371,6 +400,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
       if (mt.flags & 2) {
         // ---- finalise the segment: merge the 16 half-warp states
+        float m[HPW], l[HPW], z[HPW];
+#pragma unroll
+        for (int g = 0; g < HPW; ++g) {
+          m[g] = __shfl_sync(0xffffffffu, m_run, hbase + g);
+          l[g] = __shfl_sync(0xffffffffu, lz, hbase + g);
+          z[g] = __shfl_sync(0xffffffffu, lz, hbase + HPW + g);
+        }
 #pragma unroll
         for (int g = 0; g < HPW; ++g) {
           const float mo = __shfl_xor_sync(0xffffffffu, m[g], 16);
@@ -533,7 +569,8 @@ constexpr int decode_smem_bytes(int hpw) {
   using Cfg = DecodeTile<T, D>;
   return 1024 + Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::STAGES * (int)sizeof(TileMeta) +
          2 * Cfg::STAGES * 8 + (int)sizeof(RangeInfo) + 20 * 8 +
-         kDecConsumerWarps * hpw * part_head_floats<D>() * 4;
+         kDecConsumerWarps * hpw * part_head_floats<D>() * 4 + 16 +
+         (2 * kDecConsumerWarps * kDecRedRegion + 2 * kDecConsumerWarps * 16) * 4;
 }
 
 template <typename T, int D, int HPW>

@@ -21,9 +21,11 @@
 //    multi-stage shared-memory ring with TMA; the cache is read exactly once.
 //  * Eight consumer warps: each half-warp owns KPH keys of a tile, 16 lanes
 //    split the head dimension.  s = scale q.k and t = rho.k are partial dot
-//    products (packed fp32x2 FMA) reduced with warp shuffles; the online
-//    softmax keeps (m, l, z) per head; the two accumulators o and u per head
-//    stay in registers.
+//    products (packed fp32x2 FMA), reduced by a transpose through shared
+//    memory so that each lane ends up with one full score; the online softmax
+//    runs on those distributed scores (m, l, z per head) with a few shuffles,
+//    and the weights p and p t are broadcast back through shared memory; the
+//    two accumulators o and u per head stay in registers.
 #pragma once
 
 #include "plx_device.cuh"
@@ -33,6 +35,11 @@ namespace plx {
 constexpr int kDecConsumerWarps = 8;
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;  // + producer warp
 constexpr int kDecSmemBudget = 225 * 1024;
+// Transpose-reduction scratch per half-warp: 16 rows of 16 partial sums padded
+// to 20 floats (conflict-free 16-byte writes), and a 16-float skew between the
+// two half-warps of a warp (conflict-free column reads).
+constexpr int kDecRedRow = 20;
+constexpr int kDecRedRegion = 16 * kDecRedRow + 16;
 
 template <typename T, int D>
 struct DecodeTile {
@@ -44,7 +51,8 @@ struct DecodeTile {
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   // room left after the merge scratch of the widest head group (2 heads)
   static constexpr int RING_BUDGET = kDecSmemBudget - 2048 -
-                                     kDecConsumerWarps * 2 * (2 * D + 4) * 4;
+                                     kDecConsumerWarps * 2 * (2 * D + 4) * 4 -
+                                     (2 * kDecConsumerWarps * (kDecRedRegion + 16)) * 4;
   static constexpr int STAGES_RAW = RING_BUDGET / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 4 ? 4 : STAGES_RAW;
   static_assert(STAGES >= 2, "decode tile too large for the stage ring");

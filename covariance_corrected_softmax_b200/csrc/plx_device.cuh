@@ -312,6 +312,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The fp32 values nearest to x with 11 significant bits (fp16's precision in
+// its normal range), by Veltkamp-Dekker splitting: g = (2^13 + 1) x,
+// hi = g - (g - x).  Three packed fp32x2 operations on the FMA pipe.
+__device__ __forceinline__ float2 round_to_11_bits(float2 x) {
+  const float2 m1 = make_float2(-1.f, -1.f);
+  const float2 g = __fmul2_rn(x, make_float2(8193.f, 8193.f));
+  const float2 d = __ffma2_rn(x, m1, g);   // g - x
+  return __ffma2_rn(d, m1, g);             // g - (g - x)
+}
+
 // Round two fp32 to bf16 (nearest-even) and pack (lo in the low half).
 __device__ __forceinline__ uint32_t float2_to_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -29,8 +29,8 @@
 // convert each V tile to fp16 in place, so the PV products are fp16 x fp16 with
 // fp32 accumulation: P rounded to bf16 (8 significant bits) is not accurate
 // enough once the correction's (1 + tbar) o - u cancellation amplifies it,
-// fp16's 11 bits are.  The normalisers l = sum P and z = sum P t are summed
-// from the same rounded values the tensor core multiplies.  The running max is
+// fp16's 11 bits are.  The normalisers sum the same fp16-rounded values the
+// tensor core multiplies (rounded on the FMA pipe).  The running max is
 // rescaled lazily (only when it grows by more than 2^8, so P <= 2^8), and P t
 // carries a per-row power-of-two scale that grows only if |t| would push it
 // past fp16's range; O and U pass through registers only when either changes.
@@ -106,7 +106,7 @@ struct Bars {
 // alternately, so one named barrier per exchange suffices).
 struct Xchg {
   float2 tile[2][2][kBM];   // [slot][half][row]: (partial max, partial max |t|)
-  float4 sums[2][kBM];      // [half][row]: (l, z, l32, -)
+  float4 sums[2][kBM];      // [half][row]: (l, z, -, -)
 };
 
 template <int D, typename OutT>
@@ -316,10 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit x = unit_of(p, u);
       const int i = x.mt * kBM + r;
       // Running max m (log2 units of the scaled scores); P = 2^(s - m) <= 2^8
-      // (lazy rescaling).  Per half: l = sum P and z = sum P t 2^-eu summed
-      // from the rounded fp16 values the tensor core multiplies, and l32 = sum
-      // P unrounded (for lse).  eu (>= 0) keeps P t 2^-eu inside fp16's range.
-      float m_run = -INFINITY, l = 0.f, z = 0.f, l32 = 0.f;
+      // (lazy rescaling).  Per half: l = sum P and z = sum P t 2^-eu, each term
+      // rounded to fp16's precision first, so the normalisers match the values
+      // the tensor core multiplies.  eu (>= 0) keeps P t 2^-eu in fp16's range.
+      float m_run = -INFINITY, l = 0.f, z = 0.f;
       int eu = 0;
       for (int j = 0; j < x.n; ++j) {
         const int t = g + j, b = t & 1, st = t % kStages;
@@ -423,7 +423,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_wait_st();
           l *= alpha;
-          l32 *= alpha;
           z *= beta;
           if (resc) m_run = m_new;
           eu = eu_new;
@@ -431,27 +430,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P = 2^(s - m) as fp16 over the start of this half's S columns
         const bool live = m_run != -INFINITY;
         uint32_t pk[kHalf / 2];
-        float2 la = make_float2(0.f, 0.f), lb = la, ra = la, rb = la;
+        float2 la = make_float2(0.f, 0.f), lb = la;
+        if (live && nvis == kHalf) {
 #pragma unroll
-        for (int c = 0; c < kHalf / 2; ++c) {
-          float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), p.qscale, -m_run));
-          float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), p.qscale, -m_run));
-          if (!live || 2 * c >= nvis) p0 = 0.f;
-          if (!live || 2 * c + 1 >= nvis) p1 = 0.f;
-          sv[2 * c] = __float_as_uint(p0);
-          sv[2 * c + 1] = __float_as_uint(p1);
-          pk[c] = float2_to_f16x2(p0, p1);
-          const float2 rp = f16x2_to_float2(pk[c]);
-          if (c & 1) {
-            lb = __fadd2_rn(lb, make_float2(p0, p1));
-            rb = __fadd2_rn(rb, rp);
-          } else {
-            la = __fadd2_rn(la, make_float2(p0, p1));
-            ra = __fadd2_rn(ra, rp);
+          for (int c = 0; c < kHalf / 2; ++c) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), p.qscale, -m_run));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), p.qscale, -m_run));
+            sv[2 * c] = __float_as_uint(p0);
+            sv[2 * c + 1] = __float_as_uint(p1);
+            pk[c] = float2_to_f16x2(p0, p1);
+            const float2 rp = round_to_11_bits(make_float2(p0, p1));
+            if (c & 1)
+              lb = __fadd2_rn(lb, rp);
+            else
+              la = __fadd2_rn(la, rp);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kHalf / 2; ++c) {
+            float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), p.qscale, -m_run));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), p.qscale, -m_run));
+            if (!live || 2 * c >= nvis) p0 = 0.f;
+            if (!live || 2 * c + 1 >= nvis) p1 = 0.f;
+            sv[2 * c] = __float_as_uint(p0);
+            sv[2 * c + 1] = __float_as_uint(p1);
+            pk[c] = float2_to_f16x2(p0, p1);
+            const float2 rp = round_to_11_bits(make_float2(p0, p1));
+            if (c & 1)
+              lb = __fadd2_rn(lb, rp);
+            else
+              la = __fadd2_rn(la, rp);
           }
         }
-        l32 += (la.x + la.y) + (lb.x + lb.y);
-        l += (ra.x + ra.y) + (rb.x + rb.y);
+        l += (la.x + la.y) + (lb.x + lb.y);
         tmem_st16(lane_addr + C::COL_S + 64 * b + my_cols, pk);
         // P t 2^-eu as fp16 over the start of this half's T columns
         const float tsc = exp2f((float)-eu);
@@ -461,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float q0 = __uint_as_float(sv[2 * c]) * (__uint_as_float(tv[2 * c]) * tsc);
           const float q1 = __uint_as_float(sv[2 * c + 1]) * (__uint_as_float(tv[2 * c + 1]) * tsc);
           pk[c] = float2_to_f16x2(q0, q1);
-          const float2 rq = f16x2_to_float2(pk[c]);
+          const float2 rq = round_to_11_bits(make_float2(q0, q1));
           if (c & 1)
             zb = __fadd2_rn(zb, rq);
           else
@@ -477,13 +488,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // ---- epilogue: out = ((1 + z/l) o - u) / l, lse = ln(sum exp(scale s));
       // the halves add their sums, then each writes half of the row.
-      xch->sums[half][r] = make_float4(l, z, l32, 0.f);
+      xch->sums[half][r] = make_float4(l, z, 0.f, 0.f);
       named_bar_sync(bar_id, 64);
       {
         const float4 o = xch->sums[half ^ 1][r];
         l += o.x;
         z += o.y;
-        l32 += o.z;
       }
       const int tl = g + x.n - 1;
       if (!mbar_wait(&bars->o_done[tl & 1], (tl >> 1) & 1, abort_flag, p.err)) break;
@@ -521,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (half == 0 && p.lse && i < p.L)
-        p.lse[((size_t)x.b * p.Hq + x.h) * p.L + i] = (m_run + log2f(l32)) * 0.6931471805599453f;
+        p.lse[((size_t)x.b * p.Hq + x.h) * p.L + i] = (m_run + log2f(l)) * 0.6931471805599453f;
       tc_fence_before();
       g += x.n;
     }
