@@ -360,10 +360,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       float pw[KPH][HPW], ptw[KPH][HPW];
 #pragma unroll
       for (int kk = 0; kk < KPH; ++kk) {
-#pragma unroll
-        for (int g = 0; g < HPW; ++g) {
-          pw[kk][g] = bc[kk * NT + g];
-          ptw[kk][g] = bc[kk * NT + HPW + g];
+        if constexpr (NT == 4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(bc + kk * NT);
+          pw[kk][0] = w4.x;
+          pw[kk][1] = w4.y;
+          ptw[kk][0] = w4.z;
+          ptw[kk][1] = w4.w;
+        } else {
+          const float2 w2 = *reinterpret_cast<const float2*>(bc + kk * NT);
+          pw[kk][0] = w2.x;
+          ptw[kk][0] = w2.y;
         }
       }
 #pragma unroll

@@ -19,7 +19,7 @@
 //    combine kernel merges with the log-sum-exp rule.
 //  * One producer warp streams K and V tiles (TK keys x d) of the cache into a
 //    multi-stage shared-memory ring with TMA; the cache is read exactly once.
-//  * Eight consumer warps: each half-warp owns KPH keys of a tile, 16 lanes
+//  * Twelve consumer warps: each half-warp owns KPH keys of a tile, 16 lanes
 //    split the head dimension.  s = scale q.k and t = rho.k are partial dot
 //    products (packed fp32x2 FMA), reduced by a transpose through shared
 //    memory so that each lane ends up with one full score; the online softmax
@@ -32,7 +32,7 @@
 
 namespace plx {
 
-constexpr int kDecConsumerWarps = 8;
+constexpr int kDecConsumerWarps = 12;
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;  // + producer warp
 constexpr int kDecSmemBudget = 225 * 1024;
 // Transpose-reduction scratch per half-warp: 16 rows of 16 partial sums padded
@@ -43,8 +43,8 @@ constexpr int kDecRedRegion = 16 * kDecRedRow + 16;
 
 template <typename T, int D>
 struct DecodeTile {
-  static constexpr int KPH = 4;                                  // keys per half-warp per tile
-  static constexpr int TK = KPH * 2 * kDecConsumerWarps;         // keys per tile (64)
+  static constexpr int KPH = sizeof(T) == 2 ? 4 : 2;             // keys per half-warp per tile
+  static constexpr int TK = KPH * 2 * kDecConsumerWarps;         // keys per tile
   static constexpr int EPL = D / 16;                             // elements per lane per row
   static constexpr int ROW_BYTES = D * (int)sizeof(T);
   static constexpr int TILE_BYTES = TK * ROW_BYTES;              // one K (or V) tile
