@@ -248,6 +248,40 @@ __device__ __forceinline__ void tmem_ld2x32_sync(uint32_t ta, uint32_t tb, uint3
       : "r"(ta), "r"(tb)
       : "memory");
 }
+// Two 16-column loads (from two TMEM addresses) under one wait.
+__device__ __forceinline__ void tmem_ld2x16_sync(uint32_t ta, uint32_t tb, uint32_t (&a)[16],
+                                                 uint32_t (&b)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, "
+      "%25, %26, %27, %28, %29, %30, %31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : PLX_R8(a, 0), PLX_R8(a, 8), PLX_R8(b, 0), PLX_R8(b, 8)
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+// One 16-column load.
+__device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : PLX_R8(r, 0), PLX_R8(r, 8)
+      : "r"(taddr)
+      : "memory");
+}
+// One column from each of two TMEM addresses under one wait.
+__device__ __forceinline__ void tmem_ld2x1_sync(uint32_t ta, uint32_t tb, uint32_t& a,
+                                                uint32_t& b) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%2];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%1}, [%3];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a), "=r"(b)
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
 #undef PLX_R8
 #define PLX_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), \
                   "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
@@ -267,6 +301,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 #undef PLX_W8
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

@@ -14,26 +14,35 @@
 // tiles first):
 //   warp 0      TMA producer: Q and R tiles once per unit, K and V tiles of 64
 //               keys into a 4-stage ring (128-byte swizzled, UMMA-canonical).
-//   warp 1      MMA issuer (one thread): S = Q K^T and T = R K^T share the K
-//               tile; O += P V and U += (P o T) V share the V tile.
-//   warp 2      allocates / frees the 512 TMEM columns.
+//   warp 1      MMA issuer (one thread), in a fixed order: S = Q K^T and
+//               T = R K^T of tile j (sharing the K tile), then O += P V and
+//               U += (P o T) V of tile j-1 (sharing the V tile).
+//   warps 2-3   convert each V tile to fp16 in place (warp 2 also allocates
+//               and frees the TMEM columns).
 //   warps 4-11  softmax + epilogue: two warpgroups; thread (row, half) owns
 //               one query row (= TMEM lane) and half of each key tile's
 //               columns.  The partners of a row exchange their partial row
 //               maxima through shared memory once per tile.
-// TMEM columns: O [0, d), U [d, 2d), S buffers at 256 + 64 b, T buffers at
-// 384 + 64 b (b = tile parity): the tensor core computes S, T of tile j+1 while
-// the softmax warps turn S, T of tile j into P = 2^(s - m) and P t, which
-// they store back as fp16 over the first 32 columns of the same buffers; those
-// are the A operands (from TMEM) of the two PV products.  The softmax warps also
-// convert each V tile to fp16 in place, so the PV products are fp16 x fp16 with
-// fp32 accumulation: P rounded to bf16 (8 significant bits) is not accurate
-// enough once the correction's (1 + tbar) o - u cancellation amplifies it,
-// fp16's 11 bits are.  The normalisers sum the same fp16-rounded values the
-// tensor core multiplies (rounded on the FMA pipe).  The running max is
-// rescaled lazily (only when it grows by more than 2^8, so P <= 2^8), and P t
-// carries a per-row power-of-two scale that grows only if |t| would push it
-// past fp16's range; O and U pass through registers only when either changes.
+//
+// The PV products are fp16 x fp16 with fp32 accumulation (P rounded to bf16,
+// 8 significant bits, is not accurate enough once the correction's
+// (1 + tbar) o - u cancellation amplifies it; fp16's 11 bits are), and their B
+// operand is V with a 16-column block of fp16 ones appended, so O gains the
+// column l = sum P and U the column z = sum P t: the normalisers are summed by
+// the tensor core from exactly the fp16 values it multiplies, and the softmax
+// warps do no summing at all.  The ones block is one 8 KB array shared by all
+// ring stages: each stage's V descriptor gets its own column-block stride so
+// that its third (or, for d = 64, second) block lands on it.
+//
+// TMEM columns (d = 128): O [0, 144), U [160, 304), S [320, 384),
+// T [384, 448), P [448, 480), P t [480, 512).  S and T are single-buffered:
+// the softmax warps copy them to registers and release them at once, so the
+// tensor core computes S, T of tile j+1 while the softmax works on tile j.  P
+// and P t are fp16 pairs, the A operands (from TMEM) of the PV products.  The
+// running max is rescaled lazily (only when it grows by more than 2^8, so
+// P <= 2^8), and P t carries a per-row power-of-two scale that grows only if
+// |t| would push it past fp16's range; O and U (with their l, z columns) pass
+// through registers only when either changes.
 // Range: |v| and |rho . k| must stay below 65504 (fp16); a non-finite result
 // is reported through the device error word.
 #include "plx_launch.h"
@@ -45,32 +54,74 @@ namespace {
 constexpr int kBM = 128;      // query rows per tile = TMEM lanes
 constexpr int kBN = 64;       // keys per tile
 constexpr int kHalf = kBN / 2;  // key columns per softmax thread
-constexpr int kStages = 4;    // K/V ring depth
+constexpr int kStages = 4;    // K/V ring depth (the shared-memory layout below assumes 4)
 constexpr int kSoftWarps = 8;   // two softmax warpgroups
+constexpr int kConvWarps = 2;   // V converters
 constexpr int kThreads = (4 + kSoftWarps) * 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kOnesBytes = 8192;      // 64 keys x 64 fp16 ones, 128-byte rows
 
 template <int D>
 struct TcCfg {
+  static_assert(D == 64 || D == 128, "head dimension 64 or 128");
   static constexpr int KB = D / 64;              // 64-element (128-byte) column blocks
   static constexpr int Q_BOX = kBM * 128;        // bytes of one Q/R column block
-  static constexpr int KV_BOX = kBN * 128;       // bytes of one K/V column block
+  static constexpr int KV_BOX = kBN * 128;       // bytes of one K/V column block (8 KB)
   static constexpr int Q_BYTES = KB * Q_BOX;
   static constexpr int KV_BYTES = KB * KV_BOX;
-  static constexpr int STAGE_BYTES = 2 * KV_BYTES;
-  static constexpr int TILE_SMEM = 2 * Q_BYTES + kStages * STAGE_BYTES;
-  static constexpr uint32_t COL_O = 0, COL_U = D, COL_S = 256, COL_T = 384;
-  // S, T: bf16 Q/R (K-major) x bf16 K (K-major).  PV: fp16 P from TMEM x fp16 V
-  // (MN-major; converted in place from bf16 before use).
+  static constexpr int STAGE_BYTES = 2 * KV_BYTES;  // TMA bytes per ring stage
+  // K/V region (offsets from its start).  V stage st: block 0 at v_box(st, 0),
+  // block c at v_box(st, 0) + c * v_lbo(st); block KB is the ones array at
+  // ONES (v_box(st, 0) + KB * v_lbo(st) == ONES for every stage).
+  static constexpr int ONES = KB == 2 ? 131072 : 65536;
+  __host__ __device__ static constexpr int v_lbo(int st) { return 65536 - 8192 * st; }
+  __host__ __device__ static constexpr int v_box(int st, int c) {
+    return KB == 2 ? (c == 0 ? 16384 * st : 65536 + 8192 * st) : 8192 * st;
+  }
+  __host__ __device__ static constexpr int k_box(int st, int c) {
+    return KB == 2 ? (c == 0 ? 16384 * st + 8192 : 98304 + 8192 * st) : 32768 + 8192 * st;
+  }
+  static constexpr int KV_REGION = ONES + kOnesBytes;
+  static constexpr int TILE_SMEM = 2 * Q_BYTES + KV_REGION;
+  // TMEM columns
+  static constexpr uint32_t NPV = D + 16;                 // PV product width (V | ones)
+  static constexpr uint32_t OU = (NPV + 31) / 32 * 32;    // column stride of O and U
+  static constexpr uint32_t COL_O = 0, COL_U = OU;
+  static constexpr uint32_t COL_S = 2 * OU, COL_T = COL_S + kBN;
+  static constexpr uint32_t COL_P = COL_T + kBN, COL_PT = COL_P + kBN / 2;
+  static_assert(COL_PT + kBN / 2 <= 512, "TMEM columns");
+  // S, T: bf16 Q/R (K-major) x bf16 K (K-major).  PV: fp16 P from TMEM x fp16
+  // [V | 1] (MN-major; V converted in place from bf16 before use).
   static constexpr uint32_t IDESC_ST = umma_idesc_f16kind(kBM, kBN, false, false);
-  static constexpr uint32_t IDESC_PV = umma_idesc_f16kind(kBM, D, true, true);
+  static constexpr uint32_t IDESC_PV = umma_idesc_f16kind(kBM, NPV, true, true);
 };
 
-// Within an S (or T) buffer of 64 fp32 columns, the softmax half h writes its
-// 32 keys' fp16 values (16 packed columns) over the start of its own 32-column
-// range, so no half overwrites columns its partner has not read yet.  The PV
-// product's K-step kk (keys 16 kk .. 16 kk + 15) reads 8 packed columns at:
-__host__ __device__ constexpr uint32_t p_col(int kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
+// The shared-memory layout above places, for every stage, K and V blocks that do
+// not overlap each other, the ones array, or another stage's blocks.
+template <int D>
+constexpr bool layout_ok() {
+  using C = TcCfg<D>;
+  int lo[4 * kStages + 1] = {}, hi[4 * kStages + 1] = {}, n = 0;
+  for (int st = 0; st < kStages; ++st)
+    for (int c = 0; c < C::KB; ++c) {
+      lo[n] = C::v_box(st, c);
+      hi[n++] = C::v_box(st, c) + C::KV_BOX;
+      lo[n] = C::k_box(st, c);
+      hi[n++] = C::k_box(st, c) + C::KV_BOX;
+      if (C::v_box(st, c) != C::v_box(st, 0) + c * C::v_lbo(st)) return false;
+    }
+  lo[n] = C::ONES;
+  hi[n++] = C::ONES + (int)kOnesBytes;
+  for (int st = 0; st < kStages; ++st)
+    if (C::v_box(st, 0) + C::KB * C::v_lbo(st) != C::ONES) return false;
+  for (int a = 0; a < n; ++a) {
+    if (lo[a] % 1024 != 0 || hi[a] > C::KV_REGION) return false;
+    for (int b = a + 1; b < n; ++b)
+      if (lo[a] < hi[b] && lo[b] < hi[a]) return false;
+  }
+  return true;
+}
+static_assert(kStages == 4 && layout_ok<64>() && layout_ok<128>(), "K/V shared-memory layout");
 
 struct TcParams {
   int B, L, Hq, Hkv, G, causal, nqt, units;
@@ -96,17 +147,22 @@ __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
   return x;
 }
 
+// Tile t below is the CTA's running key-tile count over all its units.
 struct Bars {
   uint64_t q_full, q_empty, drain;
-  uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t kv_full[kStages];   // K and V of the stage landed (TMA)
+  uint64_t kv_empty[kStages];  // PV of the stage's tile completed
+  uint64_t v_ready[kStages];   // V of the stage converted to fp16 (converter warps)
+  uint64_t s_full;             // S, T of tile t computed
+  uint64_t s_free;             // S, T of tile t copied to registers (softmax warps)
+  uint64_t p_full;             // P, P t of tile t stored (softmax warps)
+  uint64_t o_done;             // PV of tile t completed
 };
 
 // Shared memory the two halves of a row exchange through (two slots, used
 // alternately, so one named barrier per exchange suffices).
 struct Xchg {
   float2 tile[2][2][kBM];   // [slot][half][row]: (partial max, partial max |t|)
-  float4 sums[2][kBM];      // [half][row]: (l, z, -, -)
 };
 
 template <int D, typename OutT>
@@ -137,13 +193,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->v_ready[s], kConvWarps);  // one arrival per converter warp
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], kSoftWarps);  // one arrival per softmax warp
-      mbar_init(&bars->o_done[b], 1);
-    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, kSoftWarps);  // one arrival per softmax warp
+    mbar_init(&bars->p_full, kSoftWarps);
+    mbar_init(&bars->o_done, 1);
     fence_mbarrier_init();
+  }
+  {
+    // the ones block appended to every V tile (fp16 1.0 = 0x3C00)
+    uint4* ones = reinterpret_cast<uint4*>(sKV + C::ONES);
+    for (int c = tid; c < (int)(kOnesBytes / 16); c += kThreads)
+      ones[c] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+    fence_proxy_async_smem();
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, 512);
@@ -179,12 +242,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          uint8_t* sK = sKV + st * C::STAGE_BYTES;
-          uint8_t* sV = sK + C::KV_BYTES;
           mbar_arrive_expect_tx(&bars->kv_full[st], C::STAGE_BYTES);
           for (int kb = 0; kb < C::KB; ++kb) {
-            tma_load_4d(sK + kb * C::KV_BOX, &kmap, &bars->kv_full[st], kb * 64, hk, j * kBN, x.b);
-            tma_load_4d(sV + kb * C::KV_BOX, &vmap, &bars->kv_full[st], kb * 64, hk, j * kBN, x.b);
+            tma_load_4d(sKV + C::k_box(st, kb), &kmap, &bars->kv_full[st], kb * 64, hk, j * kBN,
+                        x.b);
+            tma_load_4d(sKV + C::v_box(st, kb), &vmap, &bars->kv_full[st], kb * 64, hk, j * kBN,
+                        x.b);
           }
         }
         g += x.n;
@@ -199,108 +262,142 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Issues, whichever is ready first, the S/T products of the next key tile
-    // (its K tile has landed and its TMEM buffer is free, i.e. the PV products
-    // of the tile two back have been issued) or the PV products of the oldest
-    // tile whose P has been written.  The tensor core runs them in issue order.
+    // Fixed order per tile t (j-th of its unit): S/T of t once the softmax has
+    // released the S/T columns of t-1 and K of t has landed, then PV of t-1
+    // once its P is stored and its V converted.  At the first tile of a unit
+    // the PV of the previous unit's last tile goes first, since S/T of the
+    // new unit wait for its Q and R to be reloaded.  The tensor core runs the
+    // products in issue order.
     if (lane == 0) {
       // Descriptors are built once; a tile or k-step only moves the start
       // address, i.e. adds (byte offset >> 4) to the low bits.
       const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dr = smem_desc_sw128(smem_u32(sR), 16, 1024);
-      const uint64_t dk = smem_desc_sw128(smem_u32(sKV), 16, 1024);
-      const uint64_t dv = smem_desc_sw128(smem_u32(sKV) + C::KV_BYTES, C::KV_BOX, 1024);
-      int total = 0;
-      for (int u = blockIdx.x; u < p.units; u += gridDim.x) total += unit_of(p, u).n;
-      int us = blockIdx.x, js = 0, kus = 0, ns = us < p.units ? unit_of(p, us).n : 0;
-      int up = blockIdx.x, jp = 0, np = ns;
-      int ts = 0, tp = 0;
-      bool qok = false;
-      uint64_t idle_since = globaltimer_ns();
-      uint32_t spins = 0;
-      while (tp < total) {
-        bool did = false;
-        if (ts < total && ts <= tp + 1) {
-          if (js == 0 && !qok) qok = mbar_test(&bars->q_full, kus & 1);
-          const int st = ts % kStages;
-          if ((js > 0 || qok) && mbar_test(&bars->kv_full[st], (ts / kStages) & 1)) {
-            tc_fence_after();
-            const int b = ts & 1;
-            const uint64_t bk0 = dk + (uint64_t)((st * C::STAGE_BYTES) >> 4);
+      const uint64_t dkv = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+      uint64_t dv[kStages];
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint32_t off = ((k >> 2) * C::Q_BOX + (k & 3) * 32) >> 4;
-              const uint32_t koff = ((k >> 2) * C::KV_BOX + (k & 3) * 32) >> 4;
-              umma_ss(tbase + C::COL_S + 64 * b, dq + off, bk0 + koff, C::IDESC_ST,
-                      k > 0 ? 1u : 0u);
+      for (int st = 0; st < kStages; ++st)
+        dv[st] = smem_desc_sw128(smem_u32(sKV + C::v_box(st, 0)), C::v_lbo(st), 1024);
+
+      // O += P V and U += (P t) V for tile tp (first: of its unit)
+      auto issue_pv = [&](int tp, bool first) -> bool {
+        const int st = tp % kStages;
+        if (!mbar_wait(&bars->p_full, tp & 1, abort_flag, p.err)) return false;
+        if (!mbar_wait(&bars->v_ready[st], (tp / kStages) & 1, abort_flag, p.err)) return false;
+        tc_fence_after();
+        uint64_t bv = dv[0];
+#pragma unroll
+        for (int s = 1; s < kStages; ++s)
+          if (st == s) bv = dv[s];
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ts(tbase + C::COL_O, tbase + C::COL_P + 8 * kk,
+                  bv + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+                  (first && kk == 0) ? 0u : 1u);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ts(tbase + C::COL_U, tbase + C::COL_PT + 8 * kk,
+                  bv + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+                  (first && kk == 0) ? 0u : 1u);
+        umma_commit(&bars->o_done);
+        umma_commit(&bars->kv_empty[st]);
+        return true;
+      };
+
+      int t = 0, ku = 0;
+      bool ok = true, prev_first = false;
+      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ku) {
+        const int n = unit_of(p, u).n;
+        for (int j = 0; j < n; ++j, ++t) {
+          const int st = t % kStages;
+          if (j == 0) {
+            if (t > 0 && !issue_pv(t - 1, prev_first)) {
+              ok = false;
+              break;
             }
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint32_t off = ((k >> 2) * C::Q_BOX + (k & 3) * 32) >> 4;
-              const uint32_t koff = ((k >> 2) * C::KV_BOX + (k & 3) * 32) >> 4;
-              umma_ss(tbase + C::COL_T + 64 * b, dr + off, bk0 + koff, C::IDESC_ST,
-                      k > 0 ? 1u : 0u);
+            if (!mbar_wait(&bars->q_full, ku & 1, abort_flag, p.err)) {
+              ok = false;
+              break;
             }
-            umma_commit(&bars->s_full[b]);
-            if (js == ns - 1) {
-              umma_commit(&bars->q_empty);  // Q and R of this unit are no longer read
-              us += gridDim.x;
-              ++kus;
-              js = 0;
-              qok = false;
-              ns = us < p.units ? unit_of(p, us).n : 0;
-            } else {
-              ++js;
-            }
-            ++ts;
-            did = true;
-          }
-        }
-        if (!did && tp < ts && mbar_test(&bars->p_full[tp & 1], (tp >> 1) & 1)) {
-          tc_fence_after();
-          const int b = tp & 1, st = tp % kStages;
-          const uint64_t bv0 = dv + (uint64_t)((st * C::STAGE_BYTES) >> 4);
-          const bool first = jp == 0;
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ts(tbase + C::COL_O, tbase + C::COL_S + 64 * b + p_col(kk),
-                    bv0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
-                    (first && kk == 0) ? 0u : 1u);
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ts(tbase + C::COL_U, tbase + C::COL_T + 64 * b + p_col(kk),
-                    bv0 + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
-                    (first && kk == 0) ? 0u : 1u);
-          umma_commit(&bars->o_done[b]);
-          umma_commit(&bars->kv_empty[st]);
-          if (jp == np - 1) {
-            up += gridDim.x;
-            jp = 0;
-            np = up < p.units ? unit_of(p, up).n : 0;
-          } else {
-            ++jp;
-          }
-          ++tp;
-          did = true;
-        }
-        if (did) {
-          idle_since = globaltimer_ns();
-        } else if ((++spins & 255u) == 0) {
-          if (*abort_flag) break;
-          if (globaltimer_ns() - idle_since > kWaitLimitNs) {
-            record_error(p.err, kDevTimeoutMbarrier);
-            *abort_flag = 1;
+          } else if (!mbar_wait(&bars->s_free, (t - 1) & 1, abort_flag, p.err)) {
+            ok = false;
             break;
           }
+          if (!mbar_wait(&bars->kv_full[st], (t / kStages) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = ((k >> 2) * C::Q_BOX + (k & 3) * 32) >> 4;
+            const uint32_t koff = (C::k_box(st, k >> 2) + (k & 3) * 32) >> 4;
+            umma_ss(tbase + C::COL_S, dq + off, dkv + koff, C::IDESC_ST, k > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = ((k >> 2) * C::Q_BOX + (k & 3) * 32) >> 4;
+            const uint32_t koff = (C::k_box(st, k >> 2) + (k & 3) * 32) >> 4;
+            umma_ss(tbase + C::COL_T, dr + off, dkv + koff, C::IDESC_ST, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->s_full);
+          if (j == n - 1) umma_commit(&bars->q_empty);  // Q and R of this unit are no longer read
+          if (j > 0 && !issue_pv(t - 1, prev_first)) {
+            ok = false;
+            break;
+          }
+          prev_first = j == 0;
         }
       }
+      if (ok && t > 0) issue_pv(t - 1, prev_first);
       // Every MMA must have completed before the columns are released.
       umma_commit(&bars->drain);
       volatile int never = 0;
       mbar_wait(&bars->drain, 0, &never, p.err);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ V converters
+    // V of each tile -> fp16 in place (the PV products run in fp16).
+    const int ci = tid - 64;  // 0 .. 63
+    constexpr int kPer = C::KV_BOX / 16 / 64;  // 16-byte words per thread and column block
+    int g = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+      const int n = unit_of(p, u).n;
+      for (int j = 0; j < n; ++j) {
+        const int t = g + j, st = t % kStages;
+        if (!mbar_wait(&bars->kv_full[st], (t / kStages) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb) {
+          uint4* vt = reinterpret_cast<uint4*>(sKV + C::v_box(st, kb));
+          uint4 w[kPer];
+#pragma unroll
+          for (int q = 0; q < kPer; ++q) w[q] = vt[ci + 64 * q];
+#pragma unroll
+          for (int q = 0; q < kPer; ++q) {
+            float2 f;
+            f = bf16x2_to_float2(w[q].x);
+            w[q].x = float2_to_f16x2(f.x, f.y);
+            f = bf16x2_to_float2(w[q].y);
+            w[q].y = float2_to_f16x2(f.x, f.y);
+            f = bf16x2_to_float2(w[q].z);
+            w[q].z = float2_to_f16x2(f.x, f.y);
+            f = bf16x2_to_float2(w[q].w);
+            w[q].w = float2_to_f16x2(f.x, f.y);
+            vt[ci + 64 * q] = w[q];
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->v_ready[st]);
+      }
+      g += n;
+    }
+  } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int si = tid - 128;                      // 0 .. 255
     const int half = si >> 7;                      // which 32 keys of each tile
@@ -316,44 +413,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit x = unit_of(p, u);
       const int i = x.mt * kBM + r;
       // Running max m (log2 units of the scaled scores); P = 2^(s - m) <= 2^8
-      // (lazy rescaling).  Per half: l = sum P and z = sum P t 2^-eu, each term
-      // rounded to fp16's precision first, so the normalisers match the values
-      // the tensor core multiplies.  eu (>= 0) keeps P t 2^-eu in fp16's range.
-      float m_run = -INFINITY, l = 0.f, z = 0.f;
+      // (lazy rescaling).  eu (>= 0) keeps P t 2^-eu in fp16's range.
+      float m_run = -INFINITY;
       int eu = 0;
       for (int j = 0; j < x.n; ++j) {
-        const int t = g + j, b = t & 1, st = t % kStages;
-        // V of this key tile -> fp16 in place (the PV products run in fp16).
-        if (!mbar_wait(&bars->kv_full[st], (t / kStages) & 1, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
-        {
-          uint4* vt = reinterpret_cast<uint4*>(sKV + st * C::STAGE_BYTES + C::KV_BYTES);
-#pragma unroll
-          for (int c = si; c < C::KV_BYTES / 16; c += kSoftWarps * 32) {
-            uint4 w = vt[c];
-            float2 f;
-            f = bf16x2_to_float2(w.x);
-            w.x = float2_to_f16x2(f.x, f.y);
-            f = bf16x2_to_float2(w.y);
-            w.y = float2_to_f16x2(f.x, f.y);
-            f = bf16x2_to_float2(w.z);
-            w.z = float2_to_f16x2(f.x, f.y);
-            f = bf16x2_to_float2(w.w);
-            w.w = float2_to_f16x2(f.x, f.y);
-            vt[c] = w;
-          }
-          fence_proxy_async_smem();
-        }
-        if (!mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort_flag, p.err)) {
+        const int t = g + j;
+        if (!mbar_wait(&bars->s_full, t & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t sv[kHalf], tv[kHalf];
-        tmem_ld2x32_sync(lane_addr + C::COL_S + 64 * b + my_cols,
-                         lane_addr + C::COL_T + 64 * b + my_cols, sv, tv);
+        tmem_ld2x32_sync(lane_addr + C::COL_S + my_cols, lane_addr + C::COL_T + my_cols, sv, tv);
+        // S and T are in registers: the tensor core may overwrite them
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
         const int key0 = j * kBN + half * kHalf;  // first key of this half
         const int lim = p.causal ? i : p.L - 1;    // last visible key of the row
         const int nvis = max(0, min(kHalf, lim - key0 + 1));
@@ -401,17 +476,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         int eu_new = eu;
         if (tmax * exp2f((float)-eu) >= 128.f) eu_new = max(eu, (int)ceilf(log2f(tmax)) - 6);
         const bool ubump = eu_new > eu;
+        bool pv_done = j == 0;  // the previous tile's PV has completed (or belongs to the last unit)
         if (__any_sync(0xffffffffu, resc || ubump)) {
           // (the partner warp holds the same rows and takes this branch too)
-          if (j > 0 &&
-              !mbar_wait(&bars->o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag, p.err)) {
+          if (!pv_done && !mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, p.err)) {
             ok = false;
             break;
           }
+          pv_done = true;
           tc_fence_after();
           const float alpha = resc ? exp2f(m_run - m_new) : 1.f;
           const float beta = alpha * exp2f((float)(eu - eu_new));
-          const float f = half == 0 ? alpha : beta;  // half 0 rescales O, half 1 rescales U
+          const float f = half == 0 ? alpha : beta;  // half 0 rescales O (and l), half 1 U (and z)
           const uint32_t base = half == 0 ? C::COL_O : C::COL_U;
 #pragma unroll 1
           for (int cc = 0; cc < D; cc += 32) {
@@ -421,16 +497,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
             tmem_st32(lane_addr + base + cc, w);
           }
+          {
+            uint32_t w[16];
+            tmem_ld16_sync(lane_addr + base + D, w);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
+            tmem_st16(lane_addr + base + D, w);
+          }
           tmem_wait_st();
-          l *= alpha;
-          z *= beta;
           if (resc) m_run = m_new;
           eu = eu_new;
         }
-        // P = 2^(s - m) as fp16 over the start of this half's S columns
+        // P = 2^(s - m) as fp16 pairs
         const bool live = m_run != -INFINITY;
         uint32_t pk[kHalf / 2];
-        float2 la = make_float2(0.f, 0.f), lb = la;
         if (live && nvis == kHalf) {
 #pragma unroll
           for (int c = 0; c < kHalf / 2; ++c) {
@@ -439,11 +519,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[2 * c] = __float_as_uint(p0);
             sv[2 * c + 1] = __float_as_uint(p1);
             pk[c] = float2_to_f16x2(p0, p1);
-            const float2 rp = round_to_11_bits(make_float2(p0, p1));
-            if (c & 1)
-              lb = __fadd2_rn(lb, rp);
-            else
-              la = __fadd2_rn(la, rp);
           }
         } else {
 #pragma unroll
@@ -455,49 +530,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[2 * c] = __float_as_uint(p0);
             sv[2 * c + 1] = __float_as_uint(p1);
             pk[c] = float2_to_f16x2(p0, p1);
-            const float2 rp = round_to_11_bits(make_float2(p0, p1));
-            if (c & 1)
-              lb = __fadd2_rn(lb, rp);
-            else
-              la = __fadd2_rn(la, rp);
           }
         }
-        l += (la.x + la.y) + (lb.x + lb.y);
-        tmem_st16(lane_addr + C::COL_S + 64 * b + my_cols, pk);
-        // P t 2^-eu as fp16 over the start of this half's T columns
+        // the P columns are free once the previous tile's PV has completed
+        if (!pv_done && !mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st16(lane_addr + C::COL_P + my_cols / 2, pk);
+        // P t 2^-eu as fp16 pairs
         const float tsc = exp2f((float)-eu);
-        float2 za = make_float2(0.f, 0.f), zb = za;
 #pragma unroll
         for (int c = 0; c < kHalf / 2; ++c) {
           const float q0 = __uint_as_float(sv[2 * c]) * (__uint_as_float(tv[2 * c]) * tsc);
           const float q1 = __uint_as_float(sv[2 * c + 1]) * (__uint_as_float(tv[2 * c + 1]) * tsc);
           pk[c] = float2_to_f16x2(q0, q1);
-          const float2 rq = round_to_11_bits(make_float2(q0, q1));
-          if (c & 1)
-            zb = __fadd2_rn(zb, rq);
-          else
-            za = __fadd2_rn(za, rq);
         }
-        z += (za.x + za.y) + (zb.x + zb.y);
-        tmem_st16(lane_addr + C::COL_T + 64 * b + my_cols, pk);
+        tmem_st16(lane_addr + C::COL_PT + my_cols / 2, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[b]);
+        if (lane == 0) mbar_arrive(&bars->p_full);
       }
       if (!ok) break;
       // ---- epilogue: out = ((1 + z/l) o - u) / l, lse = ln(sum exp(scale s));
-      // the halves add their sums, then each writes half of the row.
-      xch->sums[half][r] = make_float4(l, z, 0.f, 0.f);
-      named_bar_sync(bar_id, 64);
-      {
-        const float4 o = xch->sums[half ^ 1][r];
-        l += o.x;
-        z += o.y;
-      }
+      // l and z are the ones-columns of O and U; each half writes half the row.
       const int tl = g + x.n - 1;
-      if (!mbar_wait(&bars->o_done[tl & 1], (tl >> 1) & 1, abort_flag, p.err)) break;
+      if (!mbar_wait(&bars->o_done, tl & 1, abort_flag, p.err)) break;
       tc_fence_after();
+      uint32_t lw, zw;
+      tmem_ld2x1_sync(lane_addr + C::COL_O + D, lane_addr + C::COL_U + D, lw, zw);
+      const float l = __uint_as_float(lw), z = __uint_as_float(zw);
       const float inv = 1.f / l;
       const float usc = exp2f((float)eu);           // undo the P t scaling
       const float c1 = (1.f + z * usc * inv) * inv;
