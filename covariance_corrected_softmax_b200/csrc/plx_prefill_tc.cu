@@ -14,15 +14,19 @@
 // tiles first):
 //   warp 0      TMA producer: Q and R tiles once per unit, K and V tiles of 64
 //               keys into a 4-stage ring (128-byte swizzled, UMMA-canonical).
-//   warp 1      MMA issuer (one thread), in a fixed order: S = Q K^T and
-//               T = R K^T of tile j (sharing the K tile), then O += P V and
-//               U += (P o T) V of tile j-1 (sharing the V tile).
-//   warps 2-3   convert each V tile to fp16 in place (warp 2 also allocates
-//               and frees the TMEM columns).
+//   warp 1      S/T issuer (one thread): S = Q K^T and T = R K^T of each key
+//               tile (sharing the K tile).
+//   warp 2      converts each V tile to fp16 in place; also allocates and
+//               frees the TMEM columns.
+//   warp 3      PV issuer (one thread): O += P V and U += (P o T) V of each
+//               key tile (sharing the V tile).
 //   warps 4-11  softmax + epilogue: two warpgroups; thread (row, half) owns
 //               one query row (= TMEM lane) and half of each key tile's
 //               columns.  The partners of a row exchange their partial row
 //               maxima through shared memory once per tile.
+// Two issuing threads in different warps keep the tensor core fed: a thread's
+// barrier wait is ordered behind its own MMAs still queued for the tensor core,
+// so a single issuer leaves the tensor core idle while it waits.
 //
 // The PV products are fp16 x fp16 with fp32 accumulation (P rounded to bf16,
 // 8 significant bits, is not accurate enough once the correction's
@@ -56,7 +60,7 @@ constexpr int kBN = 64;       // keys per tile
 constexpr int kHalf = kBN / 2;  // key columns per softmax thread
 constexpr int kStages = 4;    // K/V ring depth (the shared-memory layout below assumes 4)
 constexpr int kSoftWarps = 8;   // two softmax warpgroups
-constexpr int kConvWarps = 2;   // V converters
+constexpr int kConvWarps = 1;   // V converter
 constexpr int kThreads = (4 + kSoftWarps) * 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kOnesBytes = 8192;      // 64 keys x 64 fp16 ones, 128-byte rows
@@ -149,7 +153,7 @@ __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
 
 // Tile t below is the CTA's running key-tile count over all its units.
 struct Bars {
-  uint64_t q_full, q_empty, drain;
+  uint64_t q_full, q_empty, drain;  // drain: one arrival per issuer
   uint64_t kv_full[kStages];   // K and V of the stage landed (TMA)
   uint64_t kv_empty[kStages];  // PV of the stage's tile completed
   uint64_t v_ready[kStages];   // V of the stage converted to fp16 (converter warps)
@@ -189,11 +193,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain, 2);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
-      mbar_init(&bars->v_ready[s], kConvWarps);  // one arrival per converter warp
+      mbar_init(&bars->v_ready[s], kConvWarps);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, kSoftWarps);  // one arrival per softmax warp
@@ -261,69 +265,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Fixed order per tile t (j-th of its unit): S/T of t once the softmax has
-    // released the S/T columns of t-1 and K of t has landed, then PV of t-1
-    // once its P is stored and its V converted.  At the first tile of a unit
-    // the PV of the previous unit's last tile goes first, since S/T of the
-    // new unit wait for its Q and R to be reloaded.  The tensor core runs the
-    // products in issue order.
+    // ------------------------------------------------------------ S/T issuer
+    // S/T of tile t once the softmax has copied S/T of t-1 to registers and K
+    // of t has landed (and, at a unit's first tile, its Q and R).
     if (lane == 0) {
       // Descriptors are built once; a tile or k-step only moves the start
       // address, i.e. adds (byte offset >> 4) to the low bits.
       const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dr = smem_desc_sw128(smem_u32(sR), 16, 1024);
       const uint64_t dkv = smem_desc_sw128(smem_u32(sKV), 16, 1024);
-      uint64_t dv[kStages];
-#pragma unroll
-      for (int st = 0; st < kStages; ++st)
-        dv[st] = smem_desc_sw128(smem_u32(sKV + C::v_box(st, 0)), C::v_lbo(st), 1024);
-
-      // O += P V and U += (P t) V for tile tp (first: of its unit)
-      auto issue_pv = [&](int tp, bool first) -> bool {
-        const int st = tp % kStages;
-        if (!mbar_wait(&bars->p_full, tp & 1, abort_flag, p.err)) return false;
-        if (!mbar_wait(&bars->v_ready[st], (tp / kStages) & 1, abort_flag, p.err)) return false;
-        tc_fence_after();
-        uint64_t bv = dv[0];
-#pragma unroll
-        for (int s = 1; s < kStages; ++s)
-          if (st == s) bv = dv[s];
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tbase + C::COL_O, tbase + C::COL_P + 8 * kk,
-                  bv + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
-                  (first && kk == 0) ? 0u : 1u);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(tbase + C::COL_U, tbase + C::COL_PT + 8 * kk,
-                  bv + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
-                  (first && kk == 0) ? 0u : 1u);
-        umma_commit(&bars->o_done);
-        umma_commit(&bars->kv_empty[st]);
-        return true;
-      };
-
       int t = 0, ku = 0;
-      bool ok = true, prev_first = false;
+      bool ok = true;
       for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ku) {
         const int n = unit_of(p, u).n;
         for (int j = 0; j < n; ++j, ++t) {
           const int st = t % kStages;
-          if (j == 0) {
-            if (t > 0 && !issue_pv(t - 1, prev_first)) {
-              ok = false;
-              break;
-            }
-            if (!mbar_wait(&bars->q_full, ku & 1, abort_flag, p.err)) {
-              ok = false;
-              break;
-            }
-          } else if (!mbar_wait(&bars->s_free, (t - 1) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          if (!mbar_wait(&bars->kv_full[st], (t / kStages) & 1, abort_flag, p.err)) {
+          if ((t > 0 && !mbar_wait(&bars->s_free, (t - 1) & 1, abort_flag, p.err)) ||
+              (j == 0 && !mbar_wait(&bars->q_full, ku & 1, abort_flag, p.err)) ||
+              !mbar_wait(&bars->kv_full[st], (t / kStages) & 1, abort_flag, p.err)) {
             ok = false;
             break;
           }
@@ -342,25 +301,62 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           umma_commit(&bars->s_full);
           if (j == n - 1) umma_commit(&bars->q_empty);  // Q and R of this unit are no longer read
-          if (j > 0 && !issue_pv(t - 1, prev_first)) {
-            ok = false;
-            break;
-          }
-          prev_first = j == 0;
         }
       }
-      if (ok && t > 0) issue_pv(t - 1, prev_first);
       // Every MMA must have completed before the columns are released.
       umma_commit(&bars->drain);
       volatile int never = 0;
       mbar_wait(&bars->drain, 0, &never, p.err);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ V converters
-    // V of each tile -> fp16 in place (the PV products run in fp16).
-    const int ci = tid - 64;  // 0 .. 63
-    constexpr int kPer = C::KV_BOX / 16 / 64;  // 16-byte words per thread and column block
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ PV issuer
+    // PV of tile t once its P is stored and its V converted.  (S/T of t has
+    // completed by then, so the stage's K and V are both free after PV.)
+    if (lane == 0) {
+      uint64_t dv[kStages];
+#pragma unroll
+      for (int st = 0; st < kStages; ++st)
+        dv[st] = smem_desc_sw128(smem_u32(sKV + C::v_box(st, 0)), C::v_lbo(st), 1024);
+      int t = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+        const int n = unit_of(p, u).n;
+        for (int j = 0; j < n; ++j, ++t) {
+          const int st = t % kStages;
+          if (!mbar_wait(&bars->p_full, t & 1, abort_flag, p.err) ||
+              !mbar_wait(&bars->v_ready[st], (t / kStages) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint64_t bv = dv[0];
+#pragma unroll
+          for (int s = 1; s < kStages; ++s)
+            if (st == s) bv = dv[s];
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_ts(tbase + C::COL_O, tbase + C::COL_P + 8 * kk,
+                    bv + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+                    (j == 0 && kk == 0) ? 0u : 1u);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_ts(tbase + C::COL_U, tbase + C::COL_PT + 8 * kk,
+                    bv + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
+                    (j == 0 && kk == 0) ? 0u : 1u);
+          umma_commit(&bars->o_done);
+          umma_commit(&bars->kv_empty[st]);
+        }
+      }
+      umma_commit(&bars->drain);
+      volatile int never = 0;
+      mbar_wait(&bars->drain, 0, &never, p.err);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ V converter
+    // V of each tile -> fp16 in place (the PV products run in fp16), eight
+    // 16-byte words per thread at a time.
     int g = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
@@ -371,14 +367,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
+#pragma unroll 1
+        for (int h = 0; h < C::KV_BYTES / (16 * 32 * 8); ++h) {
+          // column block h / 2, its 256-word half h % 2
+          uint4* vt = reinterpret_cast<uint4*>(sKV + C::v_box(st, h >> 1)) + (h & 1) * 256 + lane;
+          uint4 w[8];
 #pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb) {
-          uint4* vt = reinterpret_cast<uint4*>(sKV + C::v_box(st, kb));
-          uint4 w[kPer];
+          for (int q = 0; q < 8; ++q) w[q] = vt[32 * q];
 #pragma unroll
-          for (int q = 0; q < kPer; ++q) w[q] = vt[ci + 64 * q];
-#pragma unroll
-          for (int q = 0; q < kPer; ++q) {
+          for (int q = 0; q < 8; ++q) {
             float2 f;
             f = bf16x2_to_float2(w[q].x);
             w[q].x = float2_to_f16x2(f.x, f.y);
@@ -388,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             w[q].z = float2_to_f16x2(f.x, f.y);
             f = bf16x2_to_float2(w[q].w);
             w[q].w = float2_to_f16x2(f.x, f.y);
-            vt[ci + 64 * q] = w[q];
+            vt[32 * q] = w[q];
           }
         }
         fence_proxy_async_smem();
