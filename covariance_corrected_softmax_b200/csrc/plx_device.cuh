@@ -91,6 +91,42 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Three-input max / min (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair, on the FMA pipe instead of the special-function unit.
+// Range reduction after Cody and Waite: x = n + f with n = round(x) (added to a
+// 1.5 * 2^23 bias, so n sits in the low mantissa bits) and f in [-1/2, 1/2];
+// 2^f by a degree-4 polynomial, relative-error minimax on [-1/2, 1/2] (fit by
+// exp2_poly_fit.py beside this file; max relative error 2.7e-6); 2^n added to
+// the exponent field.  Inputs are clamped to >= -32 (2^-32: below fp16's
+// smallest subnormal, which is all the callers keep) and must be <= 64.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -32.f);
+  x.y = fmaxf(x.y, -32.f);
+  const float2 bias = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const float2 y = __fadd2_rn(x, bias);
+  const float2 n = __fadd2_rn(y, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 r = make_float2(9.569985792e-03f, 9.569985792e-03f);
+  r = __ffma2_rn(r, f, make_float2(5.591785908e-02f, 5.591785908e-02f));
+  r = __ffma2_rn(r, f, make_float2(2.402474731e-01f, 2.402474731e-01f));
+  r = __ffma2_rn(r, f, make_float2(6.931217909e-01f, 6.931217909e-01f));
+  r = __ffma2_rn(r, f, make_float2(9.999992847e-01f, 9.999992847e-01f));
+  // low bits of y hold n (two's complement); << 23 moves them to the exponent
+  return make_float2(__int_as_float(__float_as_int(r.x) + (__float_as_int(y.x) << 23)),
+                     __int_as_float(__float_as_int(r.y) + (__float_as_int(y.y) << 23)));
+}
+
 // 2^x with the hardware approximation (ex2.approx.ftz.f32, about 2 ulp).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -125,6 +161,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Pull a 4-D tile into L2 ahead of its use (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c0, int c1,
+                                                   int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
 }
 
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,

@@ -64,6 +64,9 @@ constexpr int kConvWarps = 1;   // V converter
 constexpr int kThreads = (4 + kSoftWarps) * 32;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kOnesBytes = 8192;      // 64 keys x 64 fp16 ones, 128-byte rows
+// Key pairs (of a thread's 16) whose 2^x runs on the FMA pipe (exp2_poly2)
+// rather than the special-function unit, which also does the fp16 packing.
+constexpr uint32_t kPolyPairs = 0x8888u;
 
 template <int D>
 struct TcCfg {
@@ -239,6 +242,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(sQ + kb * C::Q_BOX, &qmap, &bars->q_full, kb * 64, x.h, x.mt * kBM, x.b);
           tma_load_4d(sR + kb * C::Q_BOX, &rmap, &bars->q_full, kb * 64, x.h, x.mt * kBM, x.b);
         }
+        if (u + (int)gridDim.x < p.units) {
+          // the next unit's Q and R come from L2 when the Q/R buffers free up
+          const Unit y = unit_of(p, u + gridDim.x);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            tma_prefetch_l2_4d(&qmap, kb * 64, y.h, y.mt * kBM, y.b);
+            tma_prefetch_l2_4d(&rmap, kb * 64, y.h, y.mt * kBM, y.b);
+          }
+        }
         for (int j = 0; j < x.n; ++j) {
           const int t = g + j, st = t % kStages;
           if (t >= kStages &&
@@ -413,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (lazy rescaling).  eu (>= 0) keeps P t 2^-eu in fp16's range.
       float m_run = -INFINITY;
       int eu = 0;
+      float tlim = 128.f, tsc = 1.f;  // 2^(7 + eu), 2^-eu
       for (int j = 0; j < x.n; ++j) {
         const int t = g + j;
         if (!mbar_wait(&bars->s_full, t & 1, abort_flag, p.err)) {
@@ -430,33 +442,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int lim = p.causal ? i : p.L - 1;    // last visible key of the row
         const int nvis = max(0, min(kHalf, lim - key0 + 1));
         // partial extreme of the raw scores (max if scale >= 0) and max |t|
-        float e4[4], t4[4];
+        float e2[2], t2[2];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          e4[q] = qpos ? -INFINITY : INFINITY;
-          t4[q] = 0.f;
+        for (int q = 0; q < 2; ++q) {
+          e2[q] = qpos ? -INFINITY : INFINITY;
+          t2[q] = 0.f;
         }
         if (nvis == kHalf) {
 #pragma unroll
-          for (int c = 0; c < kHalf; ++c) {
-            const float v = __uint_as_float(sv[c]);
-            e4[c & 3] = qpos ? fmaxf(e4[c & 3], v) : fminf(e4[c & 3], v);
-            t4[c & 3] = fmaxf(t4[c & 3], fabsf(__uint_as_float(tv[c])));
+          for (int c = 0; c < kHalf; c += 2) {
+            const float a = __uint_as_float(sv[c]), b = __uint_as_float(sv[c + 1]);
+            e2[(c >> 1) & 1] = qpos ? fmax3(e2[(c >> 1) & 1], a, b) : fmin3(e2[(c >> 1) & 1], a, b);
+            t2[(c >> 1) & 1] = fmax3(t2[(c >> 1) & 1], fabsf(__uint_as_float(tv[c])),
+                                     fabsf(__uint_as_float(tv[c + 1])));
           }
         } else {
 #pragma unroll
           for (int c = 0; c < kHalf; ++c) {
             const float v = __uint_as_float(sv[c]);
             if (c < nvis) {
-              e4[c & 3] = qpos ? fmaxf(e4[c & 3], v) : fminf(e4[c & 3], v);
-              t4[c & 3] = fmaxf(t4[c & 3], fabsf(__uint_as_float(tv[c])));
+              e2[c & 1] = qpos ? fmaxf(e2[c & 1], v) : fminf(e2[c & 1], v);
+              t2[c & 1] = fmaxf(t2[c & 1], fabsf(__uint_as_float(tv[c])));
             }
           }
         }
-        const float ext = qpos ? fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]))
-                               : fminf(fminf(e4[0], e4[1]), fminf(e4[2], e4[3]));
+        const float ext = qpos ? fmaxf(e2[0], e2[1]) : fminf(e2[0], e2[1]);
         float part_max = (nvis > 0) ? ext * p.qscale : -INFINITY;
-        float tmax = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
+        float tmax = fmaxf(t2[0], t2[1]);
         // combine with the partner half of the row
         xch->tile[xs & 1][half][r] = make_float2(part_max, tmax);
         named_bar_sync(bar_id, 64);
@@ -471,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (m_run == -INFINITY) m_run = m_new;
         // |P t| <= 2^8 |t|: keep |t| 2^-eu below 2^7 (P t 2^-eu below 2^15)
         int eu_new = eu;
-        if (tmax * exp2f((float)-eu) >= 128.f) eu_new = max(eu, (int)ceilf(log2f(tmax)) - 6);
+        if (tmax >= tlim) eu_new = max(eu, (int)ceilf(log2f(tmax)) - 6);
         const bool ubump = eu_new > eu;
         bool pv_done = j == 0;  // the previous tile's PV has completed (or belongs to the last unit)
         if (__any_sync(0xffffffffu, resc || ubump)) {
@@ -503,19 +515,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_wait_st();
           if (resc) m_run = m_new;
-          eu = eu_new;
+          if (ubump) {
+            eu = eu_new;
+            tlim = exp2f((float)(eu + 7));
+            tsc = exp2f((float)-eu);
+          }
         }
         // P = 2^(s - m) as fp16 pairs
         const bool live = m_run != -INFINITY;
         uint32_t pk[kHalf / 2];
         if (live && nvis == kHalf) {
+          const float2 qs2 = make_float2(p.qscale, p.qscale), nm2 = make_float2(-m_run, -m_run);
 #pragma unroll
           for (int c = 0; c < kHalf / 2; ++c) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), p.qscale, -m_run));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), p.qscale, -m_run));
-            sv[2 * c] = __float_as_uint(p0);
-            sv[2 * c + 1] = __float_as_uint(p1);
-            pk[c] = float2_to_f16x2(p0, p1);
+            const float2 xs = __ffma2_rn(
+                make_float2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), qs2, nm2);
+            const float2 pp = ((kPolyPairs >> c) & 1u)
+                                  ? exp2_poly2(xs)
+                                  : make_float2(fast_exp2(xs.x), fast_exp2(xs.y));
+            sv[2 * c] = __float_as_uint(pp.x);
+            sv[2 * c + 1] = __float_as_uint(pp.y);
+            pk[c] = float2_to_f16x2(pp.x, pp.y);
           }
         } else {
 #pragma unroll
@@ -537,12 +557,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_st16(lane_addr + C::COL_P + my_cols / 2, pk);
         // P t 2^-eu as fp16 pairs
-        const float tsc = exp2f((float)-eu);
+        {
+          const float2 tsc2 = make_float2(tsc, tsc);
 #pragma unroll
-        for (int c = 0; c < kHalf / 2; ++c) {
-          const float q0 = __uint_as_float(sv[2 * c]) * (__uint_as_float(tv[2 * c]) * tsc);
-          const float q1 = __uint_as_float(sv[2 * c + 1]) * (__uint_as_float(tv[2 * c + 1]) * tsc);
-          pk[c] = float2_to_f16x2(q0, q1);
+          for (int c = 0; c < kHalf / 2; ++c) {
+            const float2 q2 = __fmul2_rn(
+                make_float2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])),
+                __fmul2_rn(make_float2(__uint_as_float(tv[2 * c]), __uint_as_float(tv[2 * c + 1])),
+                           tsc2));
+            pk[c] = float2_to_f16x2(q2.x, q2.y);
+          }
         }
         tmem_st16(lane_addr + C::COL_PT + my_cols / 2, pk);
         tmem_wait_st();
