@@ -98,6 +98,12 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def aggregate_rate(world: int, units_per_rank: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank processes units_per_rank units per step,
+    the job takes the slowest rank's time (max_ms for all steps)."""
+    return world * units_per_rank * steps / (max_ms / 1e3)
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -412,12 +418,13 @@ def main():
     shape = W.WORKLOADS[HEADLINE]
     dec = bench_decode(plx, W, shape, args.steps, args.warmup, world, device, rank)
     ms_step = dec["ms"] / args.steps
-    tok_s = world * shape.B * args.steps / (dec["ms"] / 1e3)
+    tok_s = aggregate_rate(world, shape.B, args.steps, dec["ms"])
     gbs = dec["alg_bytes"] / (ms_step / 1e3) / 1e9
     e2e_rec = None
     if not args.no_e2e:
         e2e = bench_decode_e2e(plx, W, shape, args.steps, args.warmup, world, device, rank)
-        e2e_rec = {"value": world * shape.B * args.steps / (e2e["ms"] / 1e3), "unit": "tokens/s",
+        e2e_rec = {"value": aggregate_rate(world, shape.B, args.steps, e2e["ms"]),
+                   "unit": "tokens/s",
                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                    "ms_per_step": e2e["ms"] / args.steps}
 
@@ -434,7 +441,7 @@ def main():
                 "workload": PREFILL, "B": pshape.B, "L": pshape.L, "H_q": pshape.Hq,
                 "H_kv": pshape.Hkv, "d": pshape.d, "causal": pshape.causal, "steps": psteps,
                 "ms_per_call": pms, "tflops": tflops,
-                "tokens_per_s": world * pshape.B * pshape.L / (pms / 1e3),
+                "tokens_per_s": aggregate_rate(world, pshape.B * pshape.L, psteps, pr["ms"]),
                 "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
                              "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
                              "peak_source": f"{peak_src} bf16 dense (burst)",
