@@ -98,6 +98,19 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def gpu_index() -> int:
+    """nvidia-smi index of the current device."""
+    import torch
+    idx = torch.cuda.current_device()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            idx = int(vis.split(",")[idx])
+        except (ValueError, IndexError):
+            pass
+    return idx
+
+
 def aggregate_rate(world: int, units_per_rank: float, steps: int, max_ms: float) -> float:
     """Whole-job throughput: every rank processes units_per_rank units per step,
     the job takes the slowest rank's time (max_ms for all steps)."""
@@ -189,15 +202,8 @@ def bench_decode(plx, W, shape, steps, warmup, world, device, rank):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    gpu_idx = torch.cuda.current_device()
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    if vis:
-        try:
-            gpu_idx = int(vis.split(",")[gpu_idx])
-        except (ValueError, IndexError):
-            pass
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(gpu_idx) as clk:
+    with ClockSampler(gpu_index()) as clk:
         s.record(stream)
         for i in range(steps):
             step(warmup + i)
@@ -273,20 +279,19 @@ def cpu_baseline_decode(inp, shape, seconds: float = 12.0):
     sl = inp["seqlens"].cpu()
     rows = W.sample_rows_decode(shape.B, shape.Hq, shape.B * shape.Hq, seed=2)
     done, t_used, n = 0, 0.0, max(1, threads)
-    while done < len(rows):
-        chunk = rows[done:done + n]
+    while t_used < seconds:
+        idx = [(done + j) % len(rows) for j in range(n)]
         t0 = time.perf_counter()
-        oracle.decode(q, rho, kc, vc, sl, 1.0, rows=chunk, threads=threads)
+        oracle.decode(q, rho, kc, vc, sl, 1.0, rows=rows[idx], threads=threads)
         t_used += time.perf_counter() - t0
-        done += len(chunk)
-        if t_used >= seconds:
-            break
-        n = min(4 * n, len(rows) - done) if t_used < seconds / 4 else n
+        done += n
+        if t_used < seconds / 4:
+            n = min(4 * n, len(rows))
     rows_per_s = done / t_used
     return {"value": rows_per_s / shape.Hq, "unit": "tokens/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"{done} of {shape.B * shape.Hq} (b, h) rows of {HEADLINE} "
-                      f"(explicit fp64 covariance form), {t_used:.1f} s"}
+            "sample": f"{done} (b, h) rows (cycling over all {shape.B * shape.Hq}) of "
+                      f"{HEADLINE} (explicit fp64 covariance form), {t_used:.1f} s"}
 
 
 # ----------------------------------------------------------------------- prefill
@@ -311,15 +316,16 @@ def bench_prefill(plx, W, shape, steps, warmup, world, device, rank):
     torch.cuda.synchronize()
     barrier(world)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for i in range(steps):
-        step(i)
-    e.record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(gpu_index()) as clk:
+        s.record(stream)
+        for i in range(steps):
+            step(i)
+        e.record(stream)
+        torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world, device)
     assert plx.device_error() == 0, "prefill kernel reported a device error"
-    return {"ms": ms}
+    return {"ms": ms, "clocks": clk.summary()}
 
 
 # -------------------------------------------------------------------- reference
@@ -449,6 +455,7 @@ def main():
                              "traffic": recorded_traffic("plx_prefill_tc", PREFILL,
                                                          PREFILL_SOURCES)},
                 "gpu_launches_per_call": 1,
+                "clocks": pr["clocks"],
             }
         else:
             prefill = {"workload": PREFILL, **pr}

@@ -43,10 +43,11 @@
 // the softmax warps copy them to registers and release them at once, so the
 // tensor core computes S, T of tile j+1 while the softmax works on tile j.  P
 // and P t are fp16 pairs, the A operands (from TMEM) of the PV products.  The
-// running max is rescaled lazily (only when it grows by more than 2^8, so
-// P <= 2^8), and P t carries a per-row power-of-two scale that grows only if
-// |t| would push it past fp16's range; O and U (with their l, z columns) pass
-// through registers only when either changes.
+// running max is rescaled lazily (only when the scores exceed it by more than a
+// factor 2^8, so P <= 2^8), and P t carries a per-row power-of-two scale that
+// grows only if |t| would push it past fp16's range; O and U (with their l, z
+// columns) pass through registers only when either changes, after P and P t
+// of the tile are stored.
 // Range: |v| and |rho . k| must stay below 65504 (fp16); a non-finite result
 // is reported through the device error word.
 #include "plx_launch.h"
@@ -62,7 +63,11 @@ constexpr int kStages = 4;    // K/V ring depth (the shared-memory layout below 
 constexpr int kSoftWarps = 8;   // two softmax warpgroups
 constexpr int kConvWarps = 1;   // V converter
 constexpr int kThreads = (4 + kSoftWarps) * 32;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Lazy rescaling: the running max m moves only when a score exceeds it by more
+// than 2^kRescaleBits, so P <= 2^kRescaleBits; |t| 2^-eu is kept below
+// 2^kTBits so that |P t 2^-eu| < 2^15 stays inside fp16's range.
+constexpr int kRescaleBits = 8;
+constexpr int kTBits = 15 - kRescaleBits;
 constexpr uint32_t kOnesBytes = 8192;      // 64 keys x 64 fp16 ones, 128-byte rows
 // Key pairs (of a thread's 16) whose 2^x runs on the FMA pipe (exp2_poly2)
 // rather than the special-function unit, which also does the fp16 packing.
@@ -424,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (lazy rescaling).  eu (>= 0) keeps P t 2^-eu in fp16's range.
       float m_run = -INFINITY;
       int eu = 0;
-      float tlim = 128.f, tsc = 1.f;  // 2^(7 + eu), 2^-eu
+      float tlim = (float)(1 << kTBits), tsc = 1.f;  // 2^(kTBits + eu), 2^-eu
       for (int j = 0; j < x.n; ++j) {
         const int t = g + j;
         if (!mbar_wait(&bars->s_full, t & 1, abort_flag, p.err)) {
@@ -479,45 +484,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++xs;
         const float m_new = fmaxf(m_run, part_max);
-        const bool resc = (m_run != -INFINITY) && (m_new > m_run + kRescaleThreshold);
+        const bool resc = (m_run != -INFINITY) && (m_new > m_run + (float)kRescaleBits);
         if (m_run == -INFINITY) m_run = m_new;
-        // |P t| <= 2^8 |t|: keep |t| 2^-eu below 2^7 (P t 2^-eu below 2^15)
         int eu_new = eu;
-        if (tmax >= tlim) eu_new = max(eu, (int)ceilf(log2f(tmax)) - 6);
+        if (tmax >= tlim) eu_new = max(eu, (int)ceilf(log2f(tmax)) - (kTBits - 1));
         const bool ubump = eu_new > eu;
-        bool pv_done = j == 0;  // the previous tile's PV has completed (or belongs to the last unit)
-        if (__any_sync(0xffffffffu, resc || ubump)) {
-          // (the partner warp holds the same rows and takes this branch too)
-          if (!pv_done && !mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          pv_done = true;
-          tc_fence_after();
+        // O and U (with l, z) are rescaled below, after P and P t are stored;
+        // P and P t already use the new m and eu.  (The partner warp holds the
+        // same rows, so both warps of a row take the branch together.)
+        const bool rescale = __any_sync(0xffffffffu, resc || ubump);
+        float fr = 1.f;  // this half's factor: half 0 rescales O (and l), half 1 U (and z)
+        if (rescale) {
           const float alpha = resc ? exp2f(m_run - m_new) : 1.f;
-          const float beta = alpha * exp2f((float)(eu - eu_new));
-          const float f = half == 0 ? alpha : beta;  // half 0 rescales O (and l), half 1 U (and z)
-          const uint32_t base = half == 0 ? C::COL_O : C::COL_U;
-#pragma unroll 1
-          for (int cc = 0; cc < D; cc += 32) {
-            uint32_t w[32];
-            tmem_ld32_sync(lane_addr + base + cc, w);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
-            tmem_st32(lane_addr + base + cc, w);
-          }
-          {
-            uint32_t w[16];
-            tmem_ld16_sync(lane_addr + base + D, w);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
-            tmem_st16(lane_addr + base + D, w);
-          }
-          tmem_wait_st();
+          fr = half == 0 ? alpha : alpha * exp2f((float)(eu - eu_new));
           if (resc) m_run = m_new;
           if (ubump) {
             eu = eu_new;
-            tlim = exp2f((float)(eu + 7));
+            tlim = exp2f((float)(eu + kTBits));
             tsc = exp2f((float)-eu);
           }
         }
@@ -549,8 +532,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[c] = float2_to_f16x2(p0, p1);
           }
         }
-        // the P columns are free once the previous tile's PV has completed
-        if (!pv_done && !mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, p.err)) {
+        // the P columns (and O, U) are free once the previous tile's PV has completed
+        if (j > 0 && !mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
@@ -569,6 +552,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tmem_st16(lane_addr + C::COL_PT + my_cols / 2, pk);
+        if (rescale) {
+          const uint32_t base = lane_addr + (half == 0 ? C::COL_O : C::COL_U);
+#pragma unroll 1
+          for (int cc = 0; cc < D; cc += 64) {
+            uint32_t wa[32], wb[32];
+            tmem_ld2x32_sync(base + cc, base + cc + 32, wa, wb);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              wa[e] = __float_as_uint(__uint_as_float(wa[e]) * fr);
+              wb[e] = __float_as_uint(__uint_as_float(wb[e]) * fr);
+            }
+            tmem_st32(base + cc, wa);
+            tmem_st32(base + cc + 32, wb);
+          }
+          uint32_t w[16];
+          tmem_ld16_sync(base + D, w);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * fr);
+          tmem_st16(base + D, w);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
