@@ -180,6 +180,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     fence_mbarrier_init();
   }
   locate_range(p, TK, info, scan_ws);  // contains __syncthreads
+  // The combine kernel may be scheduled now; it waits for this grid to finish.
+  grid_dep_launch_dependents();
   if (blockIdx.x == 0 && tid == 0) reinterpret_cast<long long*>(p.ws)[0] = info->total;
 
   // Batches with an empty context produce zeros (out = 0 for an empty key set).
@@ -509,6 +511,8 @@ __global__ void __launch_bounds__(256)
     plx_decode_combine_kernel(const DecodeParams p) {
   constexpr int PF = part_floats<D>(HPW);
   constexpr int PHF = part_head_floats<D>();
+  // launched as a programmatic dependent of the main kernel: wait for it
+  grid_dep_wait();
   const float* base = p.ws + kWsHeaderFloats;
   const int c0 = blockIdx.x;
   int slot = -1;
@@ -589,7 +593,20 @@ cudaError_t launch_decode_t(const CUtensorMap& kmap, const CUtensorMap& vmap,
   kern<<<p.grid, kDecThreads, smem, stream>>>(kmap, vmap, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  plx_decode_combine_kernel<T, D, HPW><<<p.grid, 256, 0, stream>>>(p);
+  // The combine kernel is a programmatic dependent of the main kernel, so its
+  // launch overlaps the main kernel's tail (it waits for the main grid itself).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, plx_decode_combine_kernel<T, D, HPW>, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
