@@ -218,36 +218,42 @@ def bench_decode(plx, W, shape, steps, warmup, world, device, rank):
 
 
 def bench_decode_e2e(plx, W, shape, steps, warmup, world, device, rank):
-    """Same metric through the public call with host I/O every step: the new
-    token's q, rho, k, v and the lengths go host -> device from pinned memory
-    (k, v written into the cache at the last position), and out comes back."""
+    """Same metric through the public serving call with host I/O every step: the
+    new token's q, rho, k, v and the lengths (which count the new token) are
+    packed in one pinned host buffer and copied host -> device in one copy;
+    plx_decode_append writes k, v into the cache and decodes; out comes back."""
     import torch
     inp = W.make_decode(shape, seed=100 + rank, device=device, copies=3)
     B, Hq, Hkv, d = shape.B, shape.Hq, shape.Hkv, shape.d
     pos = shape.ctx - 1
-    h = {
-        "q": inp["q"].cpu().pin_memory(),
-        "rho": inp["rho"].cpu().pin_memory(),
-        "k": inp["k_cache"][:, pos].contiguous().cpu().pin_memory(),
-        "v": inp["v_cache"][:, pos].contiguous().cpu().pin_memory(),
-        "sl": inp["seqlens"].cpu().pin_memory(),
-    }
+    parts = [("q", inp["q"]), ("rho", inp["rho"]),
+             ("k", inp["k_cache"][:, pos].contiguous()), ("v", inp["v_cache"][:, pos].contiguous()),
+             ("sl", inp["seqlens"])]
+    offs, off = {}, 0
+    for name, t in parts:
+        nbytes = t.numel() * t.element_size()
+        offs[name] = (off, nbytes, t.dtype, tuple(t.shape))
+        off += (nbytes + 255) // 256 * 256
+    hbuf = torch.empty(off, dtype=torch.uint8).pin_memory()
+    for name, t in parts:
+        o, n, _, _ = offs[name]
+        hbuf[o:o + n].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
+    dbuf = torch.empty(off, dtype=torch.uint8, device=device)
+
+    def view(name):
+        o, n, dt, shp = offs[name]
+        return dbuf[o:o + n].view(dt).view(shp)
+
+    q_d, rho_d, kn_d, vn_d, sl_d = (view(n) for n in ("q", "rho", "k", "v", "sl"))
     out_h = torch.empty((B, Hq, d), dtype=inp["q"].dtype).pin_memory()
-    q_d, rho_d, sl_d = torch.empty_like(inp["q"]), torch.empty_like(inp["rho"]), \
-        torch.empty_like(inp["seqlens"])
     out_d = torch.empty_like(inp["q"])
     ws = plx.decode_workspace(B, Hq, Hkv, d, shape.S_max, device=device)
     stream = torch.cuda.current_stream()
 
     def step(i):
-        kc, vc = inp["k_caches"][i % 3], inp["v_caches"][i % 3]
-        q_d.copy_(h["q"], non_blocking=True)
-        rho_d.copy_(h["rho"], non_blocking=True)
-        kc[:, pos].copy_(h["k"], non_blocking=True)
-        vc[:, pos].copy_(h["v"], non_blocking=True)
-        sl_d.copy_(h["sl"], non_blocking=True)
-        plx.decode(q_d, rho_d, kc, vc, sl_d, softmax_scale=1.0, out=out_d, workspace=ws,
-                   stream=stream)
+        dbuf.copy_(hbuf, non_blocking=True)
+        plx.decode_append(q_d, rho_d, kn_d, vn_d, inp["k_caches"][i % 3], inp["v_caches"][i % 3],
+                          sl_d, softmax_scale=1.0, out=out_d, workspace=ws, stream=stream)
         out_h.copy_(out_d, non_blocking=True)
 
     for i in range(warmup):
@@ -262,7 +268,7 @@ def bench_decode_e2e(plx, W, shape, steps, warmup, world, device, rank):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world, device)
-    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    h2d = hbuf.numel()
     d2h = out_h.numel() * out_h.element_size()
     return {"ms": ms, "h2d": h2d, "d2h": d2h}
 
@@ -426,13 +432,15 @@ def main():
     ms_step = dec["ms"] / args.steps
     tok_s = aggregate_rate(world, shape.B, args.steps, dec["ms"])
     gbs = dec["alg_bytes"] / (ms_step / 1e3) / 1e9
-    e2e_rec = None
+    e2e_rec = None  # serving step: append the new token + decode, host I/O included
     if not args.no_e2e:
         e2e = bench_decode_e2e(plx, W, shape, args.steps, args.warmup, world, device, rank)
         e2e_rec = {"value": aggregate_rate(world, shape.B, args.steps, e2e["ms"]),
                    "unit": "tokens/s",
                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                   "ms_per_step": e2e["ms"] / args.steps}
+                   "ms_per_step": e2e["ms"] / args.steps,
+                   "call": "plx_decode_append (KV append + decode)",
+                   "gpu_launches": 3 * args.steps}
 
     prefill = None
     if not args.no_prefill:

@@ -142,10 +142,17 @@ size_t plx_decode_workspace_bytes(int B, int H_q, int H_kv, int d, int S_max) {
   return decode_ws_bytes_for(d, heads_per_pass(H_q / H_kv), sms);
 }
 
-plx_status plx_decode(const void* q, const void* rho, const void* k_cache, const void* v_cache,
-                      const int32_t* seqlens, void* out, int B, int H_q, int H_kv, int d,
-                      int S_max, plx_dtype dtype, float softmax_scale, void* workspace,
-                      size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// plx_decode, preceded (when k_new is given) by the KV-cache append of
+// plx_decode_append.  Every check runs before the first launch.
+plx_status decode_impl(const void* q, const void* rho, const void* k_new, const void* v_new,
+                       const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                       void* out, int B, int H_q, int H_kv, int d, int S_max, plx_dtype dtype,
+                       float softmax_scale, void* workspace, size_t workspace_bytes,
+                       void* stream) {
   t_last_cuda_error = 0;
   if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
   if (B < 0 || S_max < 1 || !shape_ok(H_q, H_kv, d)) return PLX_ERR_INVALID_ARGUMENT;
@@ -157,6 +164,8 @@ plx_status plx_decode(const void* q, const void* rho, const void* k_cache, const
   if (!aligned16(q) || !aligned16(rho) || !aligned16(k_cache) || !aligned16(v_cache) ||
       !aligned16(out) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
     return PLX_ERR_INVALID_ARGUMENT;
+  if ((k_new != nullptr) != (v_new != nullptr)) return PLX_ERR_INVALID_ARGUMENT;
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PLX_ERR_INVALID_ARGUMENT;
   // TMA coordinates are 32-bit; cache extents must fit.
   if ((long long)B * S_max > (1ll << 31) || (long long)B * H_q > (1 << 30))
     return PLX_ERR_UNSUPPORTED;
@@ -178,6 +187,13 @@ plx_status plx_decode(const void* q, const void* rho, const void* k_cache, const
   if (e == cudaSuccess) e = encode_rows_map(&vmap, v_cache, bf16, B, S_max, H_kv, d, tk);
   if (e != cudaSuccess) return cuda_fail(e);
 
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (k_new) {
+    e = plx::launch_kv_append(k_new, v_new, const_cast<void*>(k_cache), const_cast<void*>(v_cache),
+                              seqlens, B, H_kv, d, bf16 ? 2 : 4, S_max, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+
   plx::DecodeParams p;
   p.q = q;
   p.rho = rho;
@@ -193,9 +209,34 @@ plx_status plx_decode(const void* q, const void* rho, const void* k_cache, const
   p.qscale = softmax_scale * 1.4426950408889634f;
   p.grid = grid;
   p.err = err;
-  e = plx::launch_decode(bf16, d, kmap, vmap, p, hpw, static_cast<cudaStream_t>(stream));
+  e = plx::launch_decode(bf16, d, kmap, vmap, p, hpw, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return PLX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+plx_status plx_decode(const void* q, const void* rho, const void* k_cache, const void* v_cache,
+                      const int32_t* seqlens, void* out, int B, int H_q, int H_kv, int d,
+                      int S_max, plx_dtype dtype, float softmax_scale, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  return decode_impl(q, rho, nullptr, nullptr, k_cache, v_cache, seqlens, out, B, H_q, H_kv, d,
+                     S_max, dtype, softmax_scale, workspace, workspace_bytes, stream);
+}
+
+plx_status plx_decode_append(const void* q, const void* rho, const void* k_new,
+                             const void* v_new, void* k_cache, void* v_cache,
+                             const int32_t* seqlens, void* out, int B, int H_q, int H_kv, int d,
+                             int S_max, plx_dtype dtype, float softmax_scale, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (B > 0 && (!k_new || !v_new)) {
+    t_last_cuda_error = 0;
+    return PLX_ERR_INVALID_ARGUMENT;
+  }
+  return decode_impl(q, rho, k_new, v_new, k_cache, v_cache, seqlens, out, B, H_q, H_kv, d,
+                     S_max, dtype, softmax_scale, workspace, workspace_bytes, stream);
 }
 
 plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k, const void* v,

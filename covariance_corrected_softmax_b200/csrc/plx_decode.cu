@@ -620,6 +620,45 @@ cudaError_t launch_decode_d(const CUtensorMap& kmap, const CUtensorMap& vmap,
   }
 }
 
+// ---------------------------------------------------------------------------
+// KV-cache append: the new token's key and value rows ([B, Hkv, d]) go to
+// cache position seqlens[b] - 1 (the lengths already count the new token);
+// batches of length 0 are skipped.  One 16-byte word per thread and step; a
+// (b, kv-head) row is contiguous in both layouts.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    plx_kv_append_kernel(const uint4* k_new, const uint4* v_new, uint4* k_cache,
+                         uint4* v_cache, const int32_t* seqlens, int B, int Hkv,
+                         int words_per_row, int S_max) {
+  const long long row_words = (long long)Hkv * words_per_row;  // one batch, one position
+  const long long n = (long long)B * row_words;
+  for (long long w = (long long)blockIdx.x * blockDim.x + threadIdx.x; w < 2 * n;
+       w += (long long)gridDim.x * blockDim.x) {
+    const bool is_v = w >= n;
+    const long long x = is_v ? w - n : w;
+    const int b = (int)(x / row_words);
+    const long long rem = x - (long long)b * row_words;
+    const int len = clamp_len(seqlens[b], S_max);
+    if (len == 0) continue;
+    uint4* dst = (is_v ? v_cache : k_cache) + ((long long)b * S_max + (len - 1)) * row_words + rem;
+    *dst = (is_v ? v_new : k_new)[x];
+  }
+}
+
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                             const int32_t* seqlens, int B, int Hkv, int d, int elem_bytes,
+                             int S_max, cudaStream_t stream) {
+  const int wpr = d * elem_bytes / 16;
+  const long long words = 2ll * B * Hkv * wpr;
+  if (words == 0) return cudaSuccess;
+  long long blocks = (words + 255) / 256;
+  if (blocks > 1184) blocks = 1184;  // 8 per SM of a 148-SM part; the loop covers the rest
+  plx_kv_append_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), seqlens, B, Hkv, wpr, S_max);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode(bool bf16, int d, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const DecodeParams& p, int hpw, cudaStream_t stream) {
   if (bf16) {

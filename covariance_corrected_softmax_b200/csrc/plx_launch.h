@@ -41,6 +41,11 @@ cudaError_t launch_prefill_tc(const PrefillTcArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(bool bf16, int d, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const DecodeParams& p, int hpw, cudaStream_t stream);
 int decode_tile_keys(bool bf16, int d);
+// Writes the new token's K and V rows ([B, Hkv, d], elem_bytes per element) at
+// cache position seqlens[b] - 1 of every batch with a non-zero length.
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                             const int32_t* seqlens, int B, int Hkv, int d, int elem_bytes,
+                             int S_max, cudaStream_t stream);
 
 // TMA descriptor encoder (cuTensorMapEncodeTiled through the runtime's driver
 // entry point); null if unavailable.

@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
         L.plx_decode_workspace_bytes.restype = sz
         L.plx_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, sz, vp]
         L.plx_decode.restype = i
+        L.plx_decode_append.argtypes = [vp] * 8 + [i] * 6 + [f, vp, sz, vp]
+        L.plx_decode_append.restype = i
         L.plx_status_string.argtypes = [i]
         L.plx_status_string.restype = ctypes.c_char_p
         L.plx_last_cuda_error.argtypes = []
@@ -161,6 +163,34 @@ def decode(q: torch.Tensor, rho: torch.Tensor, k_cache: torch.Tensor, v_cache: t
                           _ptr(workspace), workspace.numel() * workspace.element_size(),
                           _stream(stream))
     _check(st, "plx_decode")
+    return out
+
+
+def decode_append(q: torch.Tensor, rho: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                  k_cache: torch.Tensor, v_cache: torch.Tensor, seqlens: torch.Tensor,
+                  softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One serving step: k_new, v_new [B, Hkv, d] are written to cache row
+    seqlens[b] - 1 (the lengths count the new token), then decode as decode()."""
+    _same(q, rho, k_new, v_new, k_cache, v_cache)
+    B, Hq, d = q.shape
+    S_max, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if rho.shape != q.shape or k_cache.shape != (B, S_max, Hkv, d) or \
+            v_cache.shape != k_cache.shape or k_new.shape != (B, Hkv, d) or \
+            v_new.shape != k_new.shape:
+        raise ValueError("shape mismatch among q, rho, k_new, v_new, k_cache, v_cache")
+    if seqlens.dtype != torch.int32 or seqlens.device != q.device or seqlens.numel() != B:
+        raise ValueError("seqlens must be int32 [B] on the same device")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, Hkv, d, S_max, device=q.device)
+    st = lib().plx_decode_append(_ptr(q), _ptr(rho), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                 _ptr(v_cache), _ptr(seqlens), _ptr(out), B, Hq, Hkv, d, S_max,
+                                 _dtype_code(q), scale, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "plx_decode_append")
     return out
 
 

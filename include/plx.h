@@ -124,6 +124,28 @@ PLX_API plx_status plx_decode(const void* q, const void* rho, const void* k_cach
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * plx_decode_append -- one serving decode step: append the new token's key and
+ * value to the KV cache, then plx_decode over the cache including it (page 3:
+ * decoding keeps a KV cache; each step adds the new token's key and value).
+ *
+ *   k_new, v_new     : [B, H_kv, d] in dtype, device, 16-byte aligned; the new
+ *                      token's key and value rows
+ *   k_cache, v_cache : [B, S_max, H_kv, d], written: for every batch with
+ *                      n = clamp(seqlens[b], 0, S_max) > 0, cache row n - 1
+ *                      becomes k_new[b] (resp. v_new[b]); no other row changes
+ *   seqlens          : lengths that already count the new token
+ * Every other argument, the workspace rule and the errors are those of
+ * plx_decode.  All checks run before anything is written; on success two
+ * writes happen in stream order: the append (one kernel), then the decode.
+ */
+PLX_API plx_status plx_decode_append(const void* q, const void* rho, const void* k_new,
+                                     const void* v_new, void* k_cache, void* v_cache,
+                                     const int32_t* seqlens, void* out, int B, int H_q,
+                                     int H_kv, int d, int S_max, plx_dtype dtype,
+                                     float softmax_scale, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * plx_decode_static_ws -- plx_decode for callers that cannot allocate device
  * memory.  The pages have no counterpart to this entry point: it is a service
  * of the library.  Callers it serves: a serving loop that must not enter the

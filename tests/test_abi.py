@@ -75,6 +75,28 @@ def test_decode_empty_batch_is_noop():
     assert _decode(B=0, q=None, k=None) == plx.PLX_OK
 
 
+def _decode_append(**kw):
+    a = dict(q=FAKE, rho=FAKE, kn=FAKE, vn=FAKE, k=FAKE, v=FAKE, sl=FAKE, out=FAKE, B=2, Hq=4,
+             Hkv=2, d=128, S=64, dtype=plx.PLX_BF16, scale=1.0, ws=FAKE, wsb=1 << 20)
+    a.update(kw)
+    return plx.lib().plx_decode_append(a["q"], a["rho"], a["kn"], a["vn"], a["k"], a["v"],
+                                       a["sl"], a["out"], a["B"], a["Hq"], a["Hkv"], a["d"],
+                                       a["S"], a["dtype"], a["scale"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(kn=None), dict(vn=None), dict(kn=FAKE + 8), dict(vn=FAKE + 4), dict(d=96),
+    dict(Hq=3, Hkv=2), dict(S=0), dict(k=None), dict(sl=FAKE + 2), dict(scale=float("nan")),
+])
+def test_decode_append_rejects(kw):
+    # argument checks come before any device work, so nothing is written
+    assert _decode_append(**kw) == INV
+
+
+def test_decode_append_empty_batch_is_noop():
+    assert _decode_append(B=0, q=None, kn=None, vn=None) == plx.PLX_OK
+
+
 @pytest.mark.parametrize("kw", [
     dict(d=32), dict(Hq=2, Hkv=3), dict(causal=2), dict(L=-1), dict(dtype=3),
     dict(scale=float("nan")), dict(q=None), dict(rho=None), dict(out=None), dict(k=FAKE + 8),
