@@ -148,11 +148,18 @@ namespace {
 
 // plx_decode, preceded (when k_new is given) by the KV-cache append of
 // plx_decode_append.  Every check runs before the first launch.
+// Paged caches (block_table != nullptr): k_cache, v_cache are the page pools
+// [num_pages, page_size, H_kv, d] and S_max = max_pages * page_size.
+struct Paging {
+  const int32_t* block_table = nullptr;
+  int num_pages = 0, page_size = 0, max_pages = 0;
+};
+
 plx_status decode_impl(const void* q, const void* rho, const void* k_new, const void* v_new,
                        const void* k_cache, const void* v_cache, const int32_t* seqlens,
                        void* out, int B, int H_q, int H_kv, int d, int S_max, plx_dtype dtype,
                        float softmax_scale, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+                       void* stream, const Paging& pg = Paging()) {
   t_last_cuda_error = 0;
   if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
   if (B < 0 || S_max < 1 || !shape_ok(H_q, H_kv, d)) return PLX_ERR_INVALID_ARGUMENT;
@@ -167,7 +174,7 @@ plx_status decode_impl(const void* q, const void* rho, const void* k_new, const 
   if ((k_new != nullptr) != (v_new != nullptr)) return PLX_ERR_INVALID_ARGUMENT;
   if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PLX_ERR_INVALID_ARGUMENT;
   // TMA coordinates are 32-bit; cache extents must fit.
-  if ((long long)B * S_max > (1ll << 31) || (long long)B * H_q > (1 << 30))
+  if ((!pg.block_table && (long long)B * S_max > (1ll << 31)) || (long long)B * H_q > (1 << 30))
     return PLX_ERR_UNSUPPORTED;
 
   const bool bf16 = dtype == PLX_BF16;
@@ -183,8 +190,15 @@ plx_status decode_impl(const void* q, const void* rho, const void* k_new, const 
   if (workspace_bytes < decode_ws_bytes_for(d, hpw, sms)) return PLX_ERR_WORKSPACE_TOO_SMALL;
 
   CUtensorMap kmap, vmap;
-  e = encode_rows_map(&kmap, k_cache, bf16, B, S_max, H_kv, d, tk);
-  if (e == cudaSuccess) e = encode_rows_map(&vmap, v_cache, bf16, B, S_max, H_kv, d, tk);
+  if (pg.block_table) {
+    // one [num_pages * page_size, H_kv, d] pool, 16-row boxes
+    const int rows = pg.num_pages * pg.page_size;
+    e = encode_rows_map(&kmap, k_cache, bf16, 1, rows, H_kv, d, 16);
+    if (e == cudaSuccess) e = encode_rows_map(&vmap, v_cache, bf16, 1, rows, H_kv, d, 16);
+  } else {
+    e = encode_rows_map(&kmap, k_cache, bf16, B, S_max, H_kv, d, tk);
+    if (e == cudaSuccess) e = encode_rows_map(&vmap, v_cache, bf16, B, S_max, H_kv, d, tk);
+  }
   if (e != cudaSuccess) return cuda_fail(e);
 
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -209,6 +223,10 @@ plx_status decode_impl(const void* q, const void* rho, const void* k_new, const 
   p.qscale = softmax_scale * 1.4426950408889634f;
   p.grid = grid;
   p.err = err;
+  p.block_table = pg.block_table;
+  p.num_pages = pg.num_pages;
+  p.page_size = pg.page_size;
+  p.max_pages = pg.max_pages;
   e = plx::launch_decode(bf16, d, kmap, vmap, p, hpw, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return PLX_OK;
@@ -224,6 +242,30 @@ plx_status plx_decode(const void* q, const void* rho, const void* k_cache, const
                       size_t workspace_bytes, void* stream) {
   return decode_impl(q, rho, nullptr, nullptr, k_cache, v_cache, seqlens, out, B, H_q, H_kv, d,
                      S_max, dtype, softmax_scale, workspace, workspace_bytes, stream);
+}
+
+plx_status plx_decode_paged(const void* q, const void* rho, const void* k_pages,
+                            const void* v_pages, const int32_t* block_table,
+                            const int32_t* seqlens, void* out, int B, int H_q, int H_kv, int d,
+                            int num_pages, int page_size, int max_pages_per_seq, plx_dtype dtype,
+                            float softmax_scale, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  t_last_cuda_error = 0;
+  if (page_size < 16 || page_size % 16 != 0 || num_pages < 1 || max_pages_per_seq < 1)
+    return PLX_ERR_INVALID_ARGUMENT;
+  if ((long long)num_pages * page_size > (1ll << 31) - 1 ||
+      (long long)max_pages_per_seq * page_size > (1ll << 31) - 1)
+    return PLX_ERR_UNSUPPORTED;
+  if (B > 0 && (!block_table || (reinterpret_cast<uintptr_t>(block_table) & 3u)))
+    return PLX_ERR_INVALID_ARGUMENT;
+  Paging pg;
+  pg.block_table = block_table;
+  pg.num_pages = num_pages;
+  pg.page_size = page_size;
+  pg.max_pages = max_pages_per_seq;
+  return decode_impl(q, rho, nullptr, nullptr, k_pages, v_pages, seqlens, out, B, H_q, H_kv, d,
+                     max_pages_per_seq * page_size, dtype, softmax_scale, workspace,
+                     workspace_bytes, stream, pg);
 }
 
 plx_status plx_decode_append(const void* q, const void* rho, const void* k_new,

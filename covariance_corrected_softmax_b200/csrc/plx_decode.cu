@@ -139,7 +139,7 @@ __device__ void locate_range(const DecodeParams& p, int TK, RangeInfo* info, lon
 // ---------------------------------------------------------------------------
 // Main decode kernel.
 // ---------------------------------------------------------------------------
-template <typename T, int D, int HPW>
+template <typename T, int D, int HPW, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, 1)
     plx_decode_splitk_kernel(const __grid_constant__ CUtensorMap kmap,
                              const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
@@ -197,20 +197,69 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   if (warp == kDecConsumerWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && t0 < t1) {
-      tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&vmap);
-      int b = info->b0;
-      int len = clamp_len(p.seqlens[b], p.S_max);
-      int nt = (len + TK - 1) / TK;
-      int seg_local = (int)(info->off0 / nt);
-      int kt = (int)(info->off0 % nt);
-      bool starts_here = (kt == 0);
-      for (long long t = t0, i = 0; t < t1; ++t, ++i) {
-        const int stage = (int)(i % STAGES);
-        if (i >= STAGES) {
-          if (!mbar_wait(&empty[stage], (uint32_t)(((i / STAGES) - 1) & 1), abort_flag, p.err)) break;
+    if constexpr (!PAGED) {
+      // contiguous cache: one lane issues one K and one V load per tile
+      if (lane == 0 && t0 < t1) {
+        tma_prefetch_desc(&kmap);
+        tma_prefetch_desc(&vmap);
+        int b = info->b0;
+        int len = clamp_len(p.seqlens[b], p.S_max);
+        int nt = (len + TK - 1) / TK;
+        int seg_local = (int)(info->off0 / nt);
+        int kt = (int)(info->off0 % nt);
+        bool starts_here = (kt == 0);
+        for (long long t = t0, i = 0; t < t1; ++t, ++i) {
+          const int stage = (int)(i % STAGES);
+          if (i >= STAGES) {
+            if (!mbar_wait(&empty[stage], (uint32_t)(((i / STAGES) - 1) & 1), abort_flag, p.err)) break;
+          }
+          TileMeta m;
+          m.b = b;
+          m.hkv = seg_local / p.nhg;
+          m.hg = seg_local % p.nhg;
+          m.kt = kt;
+          m.nvalid = min(TK, len - kt * TK);
+          m.seg = b * segs_per_b + seg_local;
+          m.flags = ((t == t0 || kt == 0) ? 1 : 0) | ((t == t1 - 1 || kt == nt - 1) ? 2 : 0) |
+                    (starts_here ? 4 : 0) | ((kt == nt - 1) ? 8 : 0);
+          m.pad = 0;
+          metas[stage] = m;
+          mbar_arrive_expect_tx(&full[stage], 2 * Cfg::TILE_BYTES);
+          uint8_t* dst = ring + stage * Cfg::STAGE_BYTES;
+          tma_load_4d(dst, &kmap, &full[stage], 0, m.hkv, kt * TK, b);
+          tma_load_4d(dst + Cfg::TILE_BYTES, &vmap, &full[stage], 0, m.hkv, kt * TK, b);
+          // advance the walk
+          if (++kt == nt) {
+            kt = 0;
+            starts_here = true;
+            if (++seg_local == segs_per_b) {
+              seg_local = 0;
+              do {
+                ++b;
+              } while (b < p.B && clamp_len(p.seqlens[b], p.S_max) == 0);
+              if (b < p.B) {
+                len = clamp_len(p.seqlens[b], p.S_max);
+                nt = (len + TK - 1) / TK;
+              }
+            }
+          }
         }
+      }
+    } else if (t0 < t1) {
+      // The same tile walk as above (batch-major over (batch, kv-head,
+      // head-group) segments, tiles of TK keys, from this CTA's first tile t0),
+      // run by every lane of the warp.
+      int b = 0, len = 0, nt = 1, seg_local = 0, kt = 0;
+      bool starts_here = false;
+      auto walk_init = [&]() {
+        b = info->b0;
+        len = clamp_len(p.seqlens[b], p.S_max);
+        nt = (len + TK - 1) / TK;
+        seg_local = (int)(info->off0 / nt);
+        kt = (int)(info->off0 % nt);
+        starts_here = (kt == 0);
+      };
+      auto tile_meta = [&](long long t) {
         TileMeta m;
         m.b = b;
         m.hkv = seg_local / p.nhg;
@@ -221,12 +270,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         m.flags = ((t == t0 || kt == 0) ? 1 : 0) | ((t == t1 - 1 || kt == nt - 1) ? 2 : 0) |
                   (starts_here ? 4 : 0) | ((kt == nt - 1) ? 8 : 0);
         m.pad = 0;
-        metas[stage] = m;
-        mbar_arrive_expect_tx(&full[stage], 2 * Cfg::TILE_BYTES);
-        uint8_t* dst = ring + stage * Cfg::STAGE_BYTES;
-        tma_load_4d(dst, &kmap, &full[stage], 0, m.hkv, kt * TK, b);
-        tma_load_4d(dst + Cfg::TILE_BYTES, &vmap, &full[stage], 0, m.hkv, kt * TK, b);
-        // advance the walk
+        return m;
+      };
+      auto walk_next = [&]() {
         if (++kt == nt) {
           kt = 0;
           starts_here = true;
@@ -241,6 +287,50 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
           }
         }
+      };
+      // Paged cache: 16-row chunks, each inside one page (page_size is a
+      // multiple of 16).  The whole warp walks the tiles; lane c looks up and
+      // loads chunk c, so the block-table reads of a tile go out together.
+      // Chunks past the length are not loaded (the consumers mask their rows);
+      // a page index outside the pool is reported and read as zeros
+      // (out-of-range TMA rows).
+      if (lane == 0) {
+        tma_prefetch_desc(&kmap);
+        tma_prefetch_desc(&vmap);
+      }
+      walk_init();
+      for (long long t = t0, i = 0; t < t1; ++t, ++i) {
+        const int stage = (int)(i % STAGES);
+        if (i >= STAGES) {
+          int okw = 1;
+          if (lane == 0)
+            okw = mbar_wait(&empty[stage], (uint32_t)(((i / STAGES) - 1) & 1), abort_flag, p.err);
+          if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+        }
+        const TileMeta m = tile_meta(t);
+        uint8_t* dst = ring + stage * Cfg::STAGE_BYTES;
+        const int nch = (m.nvalid + 15) >> 4;
+        const int c = lane;
+        int row = -16;
+        if (c < nch) {
+          const int pos = kt * TK + 16 * c;
+          const int page = p.block_table[(size_t)b * p.max_pages + pos / p.page_size];
+          if (page >= 0 && page < p.num_pages)
+            row = page * p.page_size + pos % p.page_size;
+          else
+            record_error(p.err, kDevBadArgument);
+        }
+        if (lane == 0) {
+          metas[stage] = m;
+          mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * nch * 16 * Cfg::ROW_BYTES));
+        }
+        __syncwarp();
+        if (c < nch) {
+          tma_load_4d(dst + c * 16 * Cfg::ROW_BYTES, &kmap, &full[stage], 0, m.hkv, row, 0);
+          tma_load_4d(dst + Cfg::TILE_BYTES + c * 16 * Cfg::ROW_BYTES, &vmap, &full[stage], 0,
+                      m.hkv, row, 0);
+        }
+        walk_next();
       }
     }
   } else {
@@ -587,7 +677,8 @@ template <typename T, int D, int HPW>
 cudaError_t launch_decode_t(const CUtensorMap& kmap, const CUtensorMap& vmap,
                             const DecodeParams& p, cudaStream_t stream) {
   const int smem = decode_smem_bytes<T, D>(HPW);
-  auto kern = plx_decode_splitk_kernel<T, D, HPW>;
+  auto kern = p.block_table ? plx_decode_splitk_kernel<T, D, HPW, true>
+                            : plx_decode_splitk_kernel<T, D, HPW, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<p.grid, kDecThreads, smem, stream>>>(kmap, vmap, p);

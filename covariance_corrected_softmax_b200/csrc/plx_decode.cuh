@@ -57,6 +57,7 @@ struct DecodeTile {
   static constexpr int STAGES = STAGES_RAW > 4 ? 4 : STAGES_RAW;
   static_assert(STAGES >= 2, "decode tile too large for the stage ring");
   static_assert(EPL * sizeof(T) % 8 == 0, "lane slice must be 8-byte aligned");
+  static_assert(TK % 16 == 0, "paged loads move 16-row chunks");
 };
 
 // Per-slot partial state layout (floats): header, then per head m, l, z, pad,
@@ -81,6 +82,11 @@ struct DecodeParams {
   float qscale;          // softmax scale * log2(e)
   int grid;              // number of persistent CTAs
   unsigned* err;         // device error word
+  // Paged cache (block_table != nullptr): K and V live in pools
+  // [num_pages, page_size, Hkv, D]; position j of batch b is row
+  // j % page_size of page block_table[b * max_pages + j / page_size].
+  const int32_t* block_table;
+  int num_pages, page_size, max_pages;
 };
 
 // Tile metadata written by the producer next to each stage.

@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
         L.plx_decode.restype = i
         L.plx_decode_append.argtypes = [vp] * 8 + [i] * 6 + [f, vp, sz, vp]
         L.plx_decode_append.restype = i
+        L.plx_decode_paged.argtypes = [vp] * 7 + [i] * 8 + [f, vp, sz, vp]
+        L.plx_decode_paged.restype = i
         L.plx_status_string.argtypes = [i]
         L.plx_status_string.restype = ctypes.c_char_p
         L.plx_last_cuda_error.argtypes = []
@@ -163,6 +165,39 @@ def decode(q: torch.Tensor, rho: torch.Tensor, k_cache: torch.Tensor, v_cache: t
                           _ptr(workspace), workspace.numel() * workspace.element_size(),
                           _stream(stream))
     _check(st, "plx_decode")
+    return out
+
+
+def decode_paged(q: torch.Tensor, rho: torch.Tensor, k_pages: torch.Tensor,
+                 v_pages: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor,
+                 softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode over a paged cache: k_pages, v_pages [num_pages, page_size, Hkv, d];
+    block_table int32 [B, max_pages] (device); seqlens int32 [B] (device)."""
+    _same(q, rho, k_pages, v_pages)
+    B, Hq, d = q.shape
+    num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    if rho.shape != q.shape or k_pages.shape != (num_pages, page_size, Hkv, d) or \
+            v_pages.shape != k_pages.shape:
+        raise ValueError("shape mismatch among q, rho, k_pages, v_pages")
+    if block_table.dtype != torch.int32 or block_table.device != q.device or \
+            block_table.dim() != 2 or block_table.shape[0] != B or \
+            not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 [B, max_pages] device tensor")
+    if seqlens.dtype != torch.int32 or seqlens.device != q.device or seqlens.numel() != B:
+        raise ValueError("seqlens must be int32 [B] on the same device")
+    max_pages = block_table.shape[1]
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, Hkv, d, max_pages * page_size, device=q.device)
+    st = lib().plx_decode_paged(_ptr(q), _ptr(rho), _ptr(k_pages), _ptr(v_pages),
+                                _ptr(block_table), _ptr(seqlens), _ptr(out), B, Hq, Hkv, d,
+                                num_pages, page_size, max_pages, _dtype_code(q), scale,
+                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream))
+    _check(st, "plx_decode_paged")
     return out
 
 

@@ -124,6 +124,34 @@ PLX_API plx_status plx_decode(const void* q, const void* rho, const void* k_cach
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * plx_decode_paged -- plx_decode over a paged KV cache (page 3: decoding keeps
+ * a KV cache; a serving system stores it in fixed-size pages).
+ *
+ *   k_pages, v_pages : [num_pages, page_size, H_kv, d] page pools (device,
+ *                      16-byte aligned)
+ *   block_table      : [B, max_pages_per_seq] int32, device, 4-byte aligned:
+ *                      position j of batch b is row j % page_size of page
+ *                      block_table[b * max_pages_per_seq + j / page_size]
+ *   seqlens          : [B] int32, device, clamped to [0, max_pages_per_seq *
+ *                      page_size]; entries of block_table past a sequence's
+ *                      last page are never read
+ *   page_size        : a multiple of 16 (>= 16); num_pages * page_size and
+ *                      max_pages_per_seq * page_size below 2^31
+ * q, rho, out, workspace, dtype, softmax_scale, stream: as plx_decode (the
+ * workspace size is plx_decode_workspace_bytes with S_max =
+ * max_pages_per_seq * page_size).  A page index outside [0, num_pages) read
+ * for a live position sets device error 2 (plx_device_error) and reads as
+ * zeros.  The result is bit-identical to plx_decode on the same rows stored
+ * contiguously.
+ */
+PLX_API plx_status plx_decode_paged(const void* q, const void* rho, const void* k_pages,
+                                    const void* v_pages, const int32_t* block_table,
+                                    const int32_t* seqlens, void* out, int B, int H_q,
+                                    int H_kv, int d, int num_pages, int page_size,
+                                    int max_pages_per_seq, plx_dtype dtype, float softmax_scale,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * plx_decode_append -- one serving decode step: append the new token's key and
  * value to the KV cache, then plx_decode over the cache including it (page 3:
  * decoding keeps a KV cache; each step adds the new token's key and value).

@@ -93,6 +93,33 @@ def test_decode_append_rejects(kw):
     assert _decode_append(**kw) == INV
 
 
+def _decode_paged(**kw):
+    a = dict(q=FAKE, rho=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, out=FAKE, B=2, Hq=4, Hkv=2,
+             d=128, npages=8, ps=16, maxp=4, dtype=plx.PLX_BF16, scale=1.0, ws=FAKE, wsb=1 << 20)
+    a.update(kw)
+    return plx.lib().plx_decode_paged(a["q"], a["rho"], a["kp"], a["vp"], a["bt"], a["sl"],
+                                      a["out"], a["B"], a["Hq"], a["Hkv"], a["d"], a["npages"],
+                                      a["ps"], a["maxp"], a["dtype"], a["scale"], a["ws"],
+                                      a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(ps=0), dict(ps=8), dict(ps=24), dict(npages=0), dict(maxp=0), dict(bt=None),
+    dict(bt=FAKE + 2), dict(kp=None), dict(vp=FAKE + 8), dict(d=96), dict(Hq=3, Hkv=2),
+    dict(scale=float("nan")), dict(sl=None),
+])
+def test_decode_paged_rejects(kw):
+    assert _decode_paged(**kw) == INV
+
+
+def test_decode_paged_too_large_pool_unsupported():
+    assert _decode_paged(npages=1 << 27, ps=32) == plx.PLX_ERR_UNSUPPORTED
+
+
+def test_decode_paged_empty_batch_is_noop():
+    assert _decode_paged(B=0, q=None, bt=None) == plx.PLX_OK
+
+
 def test_decode_append_empty_batch_is_noop():
     assert _decode_append(B=0, q=None, kn=None, vn=None) == plx.PLX_OK
 
