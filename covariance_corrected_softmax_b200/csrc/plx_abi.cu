@@ -244,6 +244,58 @@ plx_status plx_decode(const void* q, const void* rho, const void* k_cache, const
                      S_max, dtype, softmax_scale, workspace, workspace_bytes, stream);
 }
 
+plx_status plx_prefill_varlen(const void* q, const void* rho, const void* k, const void* v,
+                              void* out, float* lse, const int32_t* cu_seqlens, int num_seqs,
+                              int total_tokens, int max_seqlen, int causal, int H_q, int H_kv,
+                              int d, plx_dtype dtype, plx_dtype out_dtype, float softmax_scale,
+                              void* stream) {
+  t_last_cuda_error = 0;
+  if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
+  if (out_dtype != dtype && !(dtype == PLX_BF16 && out_dtype == PLX_F32))
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0 || !shape_ok(H_q, H_kv, d) ||
+      (causal != 0 && causal != 1))
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (num_seqs == 0 || total_tokens == 0 || max_seqlen == 0) return PLX_OK;
+  if (!q || !rho || !k || !v || !out || !cu_seqlens) return PLX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(rho) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (dtype != PLX_BF16) return PLX_ERR_UNSUPPORTED;  // the tensor-core path is bf16
+  if ((long long)num_seqs * H_q * ((max_seqlen + 127) / 128) > 0x7fffffffll ||
+      (long long)total_tokens * H_q > (1ll << 40) || H_q > 65535)
+    return PLX_ERR_UNSUPPORTED;
+
+  int sms = 0;
+  unsigned* err = nullptr;
+  cudaError_t e = device_info(&sms, &err);
+  if (e != cudaSuccess) return cuda_fail(e);
+  plx::PrefillTcArgs a;
+  a.q = q;
+  a.rho = rho;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.lse = lse;
+  a.B = num_seqs;
+  a.L = max_seqlen;
+  a.Hq = H_q;
+  a.Hkv = H_kv;
+  a.d = d;
+  a.causal = causal;
+  a.out_f32 = out_dtype == PLX_F32 ? 1 : 0;
+  a.scale = softmax_scale;
+  a.err = err;
+  a.num_sms = sms;
+  a.cu_seqlens = cu_seqlens;
+  a.total = total_tokens;
+  e = plx::launch_prefill_tc(a, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return PLX_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? PLX_OK : cuda_fail(e);
+}
+
 plx_status plx_decode_paged(const void* q, const void* rho, const void* k_pages,
                             const void* v_pages, const int32_t* block_table,
                             const int32_t* seqlens, void* out, int B, int H_q, int H_kv, int d,

@@ -33,6 +33,10 @@ struct PrefillTcArgs {
   float scale;
   unsigned* err;
   int num_sms;
+  // varlen (cu_seqlens != nullptr): q, rho, out [total, Hq, d], k, v [total,
+  // Hkv, d]; B sequences, L = max_seqlen; lse [Hq, total]
+  const int32_t* cu_seqlens = nullptr;
+  int total = 0;
 };
 
 cudaError_t launch_prefill_simt(const PrefillSimtParams& p, int d, cudaStream_t stream);

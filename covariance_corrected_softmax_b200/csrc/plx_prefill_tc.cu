@@ -136,17 +136,28 @@ constexpr bool layout_ok() {
 static_assert(kStages == 4 && layout_ok<64>() && layout_ok<128>(), "K/V shared-memory layout");
 
 struct TcParams {
-  int B, L, Hq, Hkv, G, causal, nqt, units;
+  int B, L, Hq, Hkv, G, causal, nqt, units;  // varlen: B = sequences, nqt from max_seqlen
   float qscale;  // softmax scale * log2(e)
   void* out;     // bf16 or fp32 (kernel template parameter)
   float* lse;
   unsigned* err;
+  const int32_t* cu_seqlens;  // varlen: sequence s is tokens [cu[s], cu[s+1])
+  int total;                  // varlen: tokens in the packed tensors
 };
 
+// A work unit: query tile mt of query head h of batch (sequence) b, with n key
+// tiles to visit.  Fixed shape: tensors [B, L, H, d]; varlen: packed [T, H, d].
 struct Unit {
-  int b, h, mt, n;  // batch, query head, query tile, key tiles
+  int b, h, mt, n;
+  int len;      // keys (= queries) of the sequence
+  int row0;     // TMA row coordinate of the sequence's position 0
+  int bc;       // TMA batch coordinate
+  int tok0;     // token index of position 0 in out
+  size_t lse0;  // lse index of position 0 of this head
+  bool bad;     // varlen: inconsistent cu_seqlens or a sequence longer than max_seqlen
 };
 
+template <bool VARLEN>
 __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
   Unit x;
   const int bh = p.B * p.Hq;
@@ -154,7 +165,29 @@ __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
   const int r = u % bh;
   x.b = r / p.Hq;
   x.h = r % p.Hq;
-  const int nk = (p.L + kBN - 1) / kBN;
+  x.bad = false;
+  if constexpr (VARLEN) {
+    const int s0 = p.cu_seqlens[x.b], s1 = p.cu_seqlens[x.b + 1];
+    const bool ok = 0 <= s0 && s0 <= s1 && s1 <= p.total;
+    x.len = ok ? s1 - s0 : 0;
+    x.row0 = ok ? s0 : 0;
+    x.bc = 0;
+    x.tok0 = x.row0;
+    x.lse0 = (size_t)x.h * p.total + x.row0;
+    const int nq = (x.len + kBM - 1) / kBM;
+    x.bad = !ok || nq > p.nqt;
+    if (x.mt >= nq) {  // no such query tile in this sequence
+      x.n = 0;
+      return x;
+    }
+  } else {
+    x.len = p.L;
+    x.row0 = 0;
+    x.bc = x.b;
+    x.tok0 = x.b * p.L;
+    x.lse0 = ((size_t)x.b * p.Hq + x.h) * p.L;
+  }
+  const int nk = (x.len + kBN - 1) / kBN;
   x.n = p.causal ? min(nk, (x.mt * kBM + kBM - 1) / kBN + 1) : nk;
   return x;
 }
@@ -177,7 +210,7 @@ struct Xchg {
   float2 tile[2][2][kBM];   // [slot][half][row]: (partial max, partial max |t|)
 };
 
-template <int D, typename OutT>
+template <int D, typename OutT, bool VARLEN>
 __global__ void __launch_bounds__(kThreads, 1)
     plx_prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                           const __grid_constant__ CUtensorMap rmap,
@@ -238,21 +271,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&vmap);
       int g = 0, ku = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ku) {
-        const Unit x = unit_of(p, u);
+      // ku counts the units with work (varlen units past a sequence's last
+      // query tile have none); every role counts them the same way
+      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+        const Unit x = unit_of<VARLEN>(p, u);
+        if constexpr (VARLEN) {
+          if (x.bad && x.mt == 0) record_error(p.err, kDevBadArgument);
+          if (x.n == 0) continue;
+        }
         const int hk = x.h / p.G;
         if (ku > 0 && !mbar_wait(&bars->q_empty, (ku - 1) & 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&bars->q_full, 2 * C::Q_BYTES);
         for (int kb = 0; kb < C::KB; ++kb) {
-          tma_load_4d(sQ + kb * C::Q_BOX, &qmap, &bars->q_full, kb * 64, x.h, x.mt * kBM, x.b);
-          tma_load_4d(sR + kb * C::Q_BOX, &rmap, &bars->q_full, kb * 64, x.h, x.mt * kBM, x.b);
+          tma_load_4d(sQ + kb * C::Q_BOX, &qmap, &bars->q_full, kb * 64, x.h,
+                      x.row0 + x.mt * kBM, x.bc);
+          tma_load_4d(sR + kb * C::Q_BOX, &rmap, &bars->q_full, kb * 64, x.h,
+                      x.row0 + x.mt * kBM, x.bc);
         }
         if (u + (int)gridDim.x < p.units) {
           // the next unit's Q and R come from L2 when the Q/R buffers free up
-          const Unit y = unit_of(p, u + gridDim.x);
-          for (int kb = 0; kb < C::KB; ++kb) {
-            tma_prefetch_l2_4d(&qmap, kb * 64, y.h, y.mt * kBM, y.b);
-            tma_prefetch_l2_4d(&rmap, kb * 64, y.h, y.mt * kBM, y.b);
+          const Unit y = unit_of<VARLEN>(p, u + gridDim.x);
+          if (y.n > 0) {
+            for (int kb = 0; kb < C::KB; ++kb) {
+              tma_prefetch_l2_4d(&qmap, kb * 64, y.h, y.row0 + y.mt * kBM, y.bc);
+              tma_prefetch_l2_4d(&rmap, kb * 64, y.h, y.row0 + y.mt * kBM, y.bc);
+            }
           }
         }
         for (int j = 0; j < x.n; ++j) {
@@ -264,13 +307,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&bars->kv_full[st], C::STAGE_BYTES);
           for (int kb = 0; kb < C::KB; ++kb) {
-            tma_load_4d(sKV + C::k_box(st, kb), &kmap, &bars->kv_full[st], kb * 64, hk, j * kBN,
-                        x.b);
-            tma_load_4d(sKV + C::v_box(st, kb), &vmap, &bars->kv_full[st], kb * 64, hk, j * kBN,
-                        x.b);
+            tma_load_4d(sKV + C::k_box(st, kb), &kmap, &bars->kv_full[st], kb * 64, hk,
+                        x.row0 + j * kBN, x.bc);
+            tma_load_4d(sKV + C::v_box(st, kb), &vmap, &bars->kv_full[st], kb * 64, hk,
+                        x.row0 + j * kBN, x.bc);
           }
         }
         g += x.n;
+        ++ku;
       }
       if (*abort_flag) {
         // let copies already in flight land before the CTA's memory is released
@@ -292,8 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dkv = smem_desc_sw128(smem_u32(sKV), 16, 1024);
       int t = 0, ku = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++ku) {
-        const int n = unit_of(p, u).n;
+      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+        const int n = unit_of<VARLEN>(p, u).n;
+        if (n == 0) continue;
         for (int j = 0; j < n; ++j, ++t) {
           const int st = t % kStages;
           if ((t > 0 && !mbar_wait(&bars->s_free, (t - 1) & 1, abort_flag, p.err)) ||
@@ -318,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&bars->s_full);
           if (j == n - 1) umma_commit(&bars->q_empty);  // Q and R of this unit are no longer read
         }
+        ++ku;
       }
       // Every MMA must have completed before the columns are released.
       umma_commit(&bars->drain);
@@ -337,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-        const int n = unit_of(p, u).n;
+        const int n = unit_of<VARLEN>(p, u).n;
         for (int j = 0; j < n; ++j, ++t) {
           const int st = t % kStages;
           if (!mbar_wait(&bars->p_full, t & 1, abort_flag, p.err) ||
@@ -376,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-      const int n = unit_of(p, u).n;
+      const int n = unit_of<VARLEN>(p, u).n;
       for (int j = 0; j < n; ++j) {
         const int t = g + j, st = t % kStages;
         if (!mbar_wait(&bars->kv_full[st], (t / kStages) & 1, abort_flag, p.err)) {
@@ -423,7 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0, xs = 0;
     bool ok = true, finite = true;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-      const Unit x = unit_of(p, u);
+      const Unit x = unit_of<VARLEN>(p, u);
+      if (x.n == 0) continue;  // (varlen) no such query tile
       const int i = x.mt * kBM + r;
       // Running max m (log2 units of the scaled scores); P = 2^(s - m) <= 2^8
       // (lazy rescaling).  eu (>= 0) keeps P t 2^-eu in fp16's range.
@@ -444,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free);
         const int key0 = j * kBN + half * kHalf;  // first key of this half
-        const int lim = p.causal ? i : p.L - 1;    // last visible key of the row
+        const int lim = p.causal ? i : x.len - 1;  // last visible key of the row
         const int nvis = max(0, min(kHalf, lim - key0 + 1));
         // partial extreme of the raw scores (max if scale >= 0) and max |t|
         float e2[2], t2[2];
@@ -590,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float usc = exp2f((float)eu);           // undo the P t scaling
       const float c1 = (1.f + z * usc * inv) * inv;
       const float cu = usc * inv;
-      OutT* orow = static_cast<OutT*>(p.out) + (((size_t)x.b * p.L + i) * p.Hq + x.h) * D;
+      OutT* orow = static_cast<OutT*>(p.out) + (((size_t)x.tok0 + i) * p.Hq + x.h) * D;
 #pragma unroll 1
       for (int cc = half * (D / 2); cc < (half + 1) * (D / 2); cc += 32) {
         uint32_t ov[32], uv[32];
@@ -601,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           a[e] = __uint_as_float(ov[e]) * c1 - __uint_as_float(uv[e]) * cu;
           finite = finite && isfinite(a[e]);
         }
-        if (i < p.L) {
+        if (i < x.len) {
           if constexpr (sizeof(OutT) == 2) {
             uint4* dst = reinterpret_cast<uint4*>(orow + cc);
 #pragma unroll
@@ -618,8 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (half == 0 && p.lse && i < p.L)
-        p.lse[((size_t)x.b * p.Hq + x.h) * p.L + i] = (m_run + log2f(l)) * 0.6931471805599453f;
+      if (half == 0 && p.lse && i < x.len)
+        p.lse[x.lse0 + i] = (m_run + log2f(l)) * 0.6931471805599453f;
       tc_fence_before();
       g += x.n;
     }
@@ -650,14 +697,16 @@ cudaError_t encode_sw128(CUtensorMap* map, const void* base, int B, int S, int H
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D, typename OutT>
+template <int D, typename OutT, bool VARLEN>
 cudaError_t launch_d(const PrefillTcArgs& a, cudaStream_t stream) {
   using C = TcCfg<D>;
   CUtensorMap qm, rm, km, vm;
-  cudaError_t e = encode_sw128(&qm, a.q, a.B, a.L, a.Hq, D, kBM);
-  if (e == cudaSuccess) e = encode_sw128(&rm, a.rho, a.B, a.L, a.Hq, D, kBM);
-  if (e == cudaSuccess) e = encode_sw128(&km, a.k, a.B, a.L, a.Hkv, D, kBN);
-  if (e == cudaSuccess) e = encode_sw128(&vm, a.v, a.B, a.L, a.Hkv, D, kBN);
+  // varlen: the packed [T, H, d] tensors as one batch of T rows
+  const int mb = VARLEN ? 1 : a.B, ms = VARLEN ? a.total : a.L;
+  cudaError_t e = encode_sw128(&qm, a.q, mb, ms, a.Hq, D, kBM);
+  if (e == cudaSuccess) e = encode_sw128(&rm, a.rho, mb, ms, a.Hq, D, kBM);
+  if (e == cudaSuccess) e = encode_sw128(&km, a.k, mb, ms, a.Hkv, D, kBN);
+  if (e == cudaSuccess) e = encode_sw128(&vm, a.v, mb, ms, a.Hkv, D, kBN);
   if (e != cudaSuccess) return e;
   TcParams p;
   p.B = a.B;
@@ -674,8 +723,10 @@ cudaError_t launch_d(const PrefillTcArgs& a, cudaStream_t stream) {
   p.out = a.out;
   p.lse = a.lse;
   p.err = a.err;
+  p.cu_seqlens = a.cu_seqlens;
+  p.total = a.total;
   const int smem = 1024 + C::TILE_SMEM + (int)sizeof(Xchg) + (int)sizeof(Bars) + 16;
-  auto kern = plx_prefill_tc_kernel<D, OutT>;
+  auto kern = plx_prefill_tc_kernel<D, OutT, VARLEN>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = (int)(units < a.num_sms ? units : a.num_sms);
@@ -685,12 +736,19 @@ cudaError_t launch_d(const PrefillTcArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_prefill_tc(const PrefillTcArgs& a, cudaStream_t stream) {
+template <bool VARLEN>
+cudaError_t launch_v(const PrefillTcArgs& a, cudaStream_t stream) {
   if (a.d == 128)
-    return a.out_f32 ? launch_d<128, float>(a, stream) : launch_d<128, __nv_bfloat16>(a, stream);
+    return a.out_f32 ? launch_d<128, float, VARLEN>(a, stream)
+                     : launch_d<128, __nv_bfloat16, VARLEN>(a, stream);
   if (a.d == 64)
-    return a.out_f32 ? launch_d<64, float>(a, stream) : launch_d<64, __nv_bfloat16>(a, stream);
+    return a.out_f32 ? launch_d<64, float, VARLEN>(a, stream)
+                     : launch_d<64, __nv_bfloat16, VARLEN>(a, stream);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill_tc(const PrefillTcArgs& a, cudaStream_t stream) {
+  return a.cu_seqlens ? launch_v<true>(a, stream) : launch_v<false>(a, stream);
 }
 
 }  // namespace plx

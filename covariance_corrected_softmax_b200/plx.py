@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
         L.plx_decode_append.restype = i
         L.plx_decode_paged.argtypes = [vp] * 7 + [i] * 8 + [f, vp, sz, vp]
         L.plx_decode_paged.restype = i
+        L.plx_prefill_varlen.argtypes = [vp] * 7 + [i] * 9 + [f, vp]
+        L.plx_prefill_varlen.restype = i
         L.plx_status_string.argtypes = [i]
         L.plx_status_string.restype = ctypes.c_char_p
         L.plx_last_cuda_error.argtypes = []
@@ -125,6 +127,37 @@ def prefill(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch.Tensor
                                _ptr(lse) if return_lse else None, int(bool(causal)), B, L, Hq,
                                Hkv, d, _dtype_code(q), _dtype_code(out), scale, _stream(stream))
     _check(st, "plx_prefill_fwd")
+    return out, (lse if return_lse else None)
+
+
+def prefill_varlen(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                   cu_seqlens: torch.Tensor, max_seqlen: int, causal: bool = True,
+                   softmax_scale: Optional[float] = None, return_lse: bool = True,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   stream=None, out_dtype: Optional[torch.dtype] = None
+                   ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Packed variable-length forward: q, rho [T, Hq, d]; k, v [T, Hkv, d];
+    cu_seqlens int32 [num_seqs + 1] on the device; max_seqlen >= every length.
+    Returns (out [T, Hq, d], lse [Hq, T] fp32 or None)."""
+    _same(q, rho, k, v)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if rho.shape != q.shape or k.shape != (T, Hkv, d) or v.shape != k.shape:
+        raise ValueError("shape mismatch among q, rho, k, v")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != q.device or \
+            cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous int32 [num_seqs + 1] device tensor")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
+    st = lib().plx_prefill_varlen(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out),
+                                  _ptr(lse) if return_lse else None, _ptr(cu_seqlens),
+                                  cu_seqlens.numel() - 1, T, int(max_seqlen), int(bool(causal)),
+                                  Hq, Hkv, d, _dtype_code(q), _dtype_code(out), scale,
+                                  _stream(stream))
+    _check(st, "plx_prefill_varlen")
     return out, (lse if return_lse else None)
 
 

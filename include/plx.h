@@ -96,6 +96,31 @@ PLX_API plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k
                                    plx_dtype out_dtype, float softmax_scale, void* stream);
 
 /*
+ * plx_prefill_varlen -- plx_prefill_fwd over sequences of different lengths
+ * packed along the token axis (same operator per sequence; page 1 opening
+ * formula and section 1.3).
+ *
+ *   q, rho, out : [total_tokens, H_q, d]   k, v : [total_tokens, H_kv, d]
+ *   lse         : [H_q, total_tokens] fp32, natural log; may be NULL
+ *   cu_seqlens  : [num_seqs + 1] int32, device, 4-byte aligned: sequence s is
+ *                 tokens cu_seqlens[s] .. cu_seqlens[s+1]-1 (0 = cu[0] <= cu[1]
+ *                 <= ... <= cu[num_seqs] <= total_tokens)
+ *   max_seqlen  : an upper bound on every sequence's length (host value)
+ * Other arguments as plx_prefill_fwd; a sequence attends only to its own keys
+ * (causal: to its own keys up to the query's position).  PLX_BF16 only
+ * (PLX_F32 returns PLX_ERR_UNSUPPORTED).  Inconsistent cu_seqlens or a
+ * sequence longer than max_seqlen set device error 2 (plx_device_error); rows
+ * of such a sequence beyond max_seqlen are not written.  Each sequence's rows
+ * equal plx_prefill_fwd on that sequence alone (B = 1, L = its length).
+ */
+PLX_API plx_status plx_prefill_varlen(const void* q, const void* rho, const void* k,
+                                      const void* v, void* out, float* lse,
+                                      const int32_t* cu_seqlens, int num_seqs,
+                                      int total_tokens, int max_seqlen, int causal, int H_q,
+                                      int H_kv, int d, plx_dtype dtype, plx_dtype out_dtype,
+                                      float softmax_scale, void* stream);
+
+/*
  * plx_decode_workspace_bytes -- device workspace that plx_decode needs for the
  * given shape on the CURRENT device (it depends on the device's SM count).
  * Returns 0 for an invalid shape.

@@ -133,6 +133,31 @@ def test_prefill_rejects(kw):
     assert _prefill(**kw) == INV
 
 
+def _prefill_varlen(**kw):
+    a = dict(q=FAKE, rho=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=None, cu=FAKE, n=3, T=300, maxs=128,
+             causal=1, Hq=4, Hkv=2, d=128, dtype=plx.PLX_BF16, out_dtype=None, scale=0.1)
+    a.update(kw)
+    od = a["dtype"] if a["out_dtype"] is None else a["out_dtype"]
+    return plx.lib().plx_prefill_varlen(a["q"], a["rho"], a["k"], a["v"], a["out"], a["lse"],
+                                        a["cu"], a["n"], a["T"], a["maxs"], a["causal"], a["Hq"],
+                                        a["Hkv"], a["d"], a["dtype"], od, a["scale"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(n=-1), dict(T=-1), dict(maxs=-1), dict(d=80), dict(Hq=3, Hkv=2), dict(causal=3),
+    dict(cu=None), dict(cu=FAKE + 2), dict(q=None), dict(k=FAKE + 8), dict(lse=FAKE + 1),
+    dict(scale=float("nan")), dict(out_dtype=5),
+])
+def test_prefill_varlen_rejects(kw):
+    assert _prefill_varlen(**kw) == INV
+
+
+def test_prefill_varlen_fp32_unsupported_and_empty_noop():
+    assert _prefill_varlen(dtype=plx.PLX_F32) == plx.PLX_ERR_UNSUPPORTED
+    assert _prefill_varlen(n=0, q=None) == plx.PLX_OK
+    assert _prefill_varlen(T=0, q=None) == plx.PLX_OK
+
+
 def test_prefill_empty_is_noop():
     assert _prefill(B=0, q=None) == plx.PLX_OK
     assert _prefill(L=0, q=None) == plx.PLX_OK
