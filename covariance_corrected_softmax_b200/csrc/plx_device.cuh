@@ -168,7 +168,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), plain (no multicast) tile loads into this CTA's
+// TMA (cp.async.bulk.tensor), plain tile loads into this CTA's
 // shared memory, completing on an mbarrier with a transaction count.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
