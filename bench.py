@@ -459,6 +459,10 @@ def main():
                 "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
                              "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
                              "peak_source": f"{peak_src} bf16 dense (burst)",
+                             # the leg runs `psteps` calls back to back (a long loop under
+                             # the power cap): the sustained GEMM figure, for comparison
+                             "peak_sustained": peaks["bf16_tflops_sustained"],
+                             "frac_sustained": tflops / peaks["bf16_tflops_sustained"],
                              "flops_per_call": pshape.flops(),
                              "traffic": recorded_traffic("plx_prefill_tc", PREFILL,
                                                          PREFILL_SOURCES)},
