@@ -159,17 +159,18 @@ plx_status decode_impl(const void* q, const void* rho, const void* k_new, const 
                        const void* k_cache, const void* v_cache, const int32_t* seqlens,
                        void* out, int B, int H_q, int H_kv, int d, int S_max, plx_dtype dtype,
                        float softmax_scale, void* workspace, size_t workspace_bytes,
-                       void* stream, const Paging& pg = Paging()) {
+                       void* stream, const Paging& pg = Paging(), float* state = nullptr) {
   t_last_cuda_error = 0;
   if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
   if (B < 0 || S_max < 1 || !shape_ok(H_q, H_kv, d)) return PLX_ERR_INVALID_ARGUMENT;
   if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
     return PLX_ERR_INVALID_ARGUMENT;
   if (B == 0) return PLX_OK;
-  if (!q || !rho || !k_cache || !v_cache || !seqlens || !out || !workspace)
+  if (!q || !rho || !k_cache || !v_cache || !seqlens || !(out || state) || !workspace)
     return PLX_ERR_INVALID_ARGUMENT;
   if (!aligned16(q) || !aligned16(rho) || !aligned16(k_cache) || !aligned16(v_cache) ||
-      !aligned16(out) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+      !aligned16(out) || !aligned16(state) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u))
     return PLX_ERR_INVALID_ARGUMENT;
   if ((k_new != nullptr) != (v_new != nullptr)) return PLX_ERR_INVALID_ARGUMENT;
   if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PLX_ERR_INVALID_ARGUMENT;
@@ -227,6 +228,7 @@ plx_status decode_impl(const void* q, const void* rho, const void* k_new, const 
   p.num_pages = pg.num_pages;
   p.page_size = pg.page_size;
   p.max_pages = pg.max_pages;
+  p.state = state;
   e = plx::launch_decode(bf16, d, kmap, vmap, p, hpw, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return PLX_OK;
@@ -293,6 +295,33 @@ plx_status plx_prefill_varlen(const void* q, const void* rho, const void* k, con
   a.total = total_tokens;
   e = plx::launch_prefill_tc(a, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return PLX_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? PLX_OK : cuda_fail(e);
+}
+
+plx_status plx_decode_state(const void* q, const void* rho, const void* k_cache,
+                            const void* v_cache, const int32_t* seqlens, float* state, int B,
+                            int H_q, int H_kv, int d, int S_max, plx_dtype dtype,
+                            float softmax_scale, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (B > 0 && !state) {
+    t_last_cuda_error = 0;
+    return PLX_ERR_INVALID_ARGUMENT;
+  }
+  return decode_impl(q, rho, nullptr, nullptr, k_cache, v_cache, seqlens, nullptr, B, H_q, H_kv,
+                     d, S_max, dtype, softmax_scale, workspace, workspace_bytes, stream, Paging(),
+                     state);
+}
+
+plx_status plx_merge_states(const float* states, int R, void* out, int B, int H_q, int d,
+                            plx_dtype out_dtype, void* stream) {
+  t_last_cuda_error = 0;
+  if (out_dtype != PLX_F32 && out_dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
+  if (R < 1 || B < 0 || H_q < 1 || (d != 64 && d != 128)) return PLX_ERR_INVALID_ARGUMENT;
+  if (B == 0) return PLX_OK;
+  if (!states || !out || !aligned16(states) || !aligned16(out)) return PLX_ERR_INVALID_ARGUMENT;
+  const cudaError_t e = plx::launch_merge_states(states, R, (long long)B * H_q, out, d,
+                                                 out_dtype == PLX_BF16,
+                                                 static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PLX_OK : cuda_fail(e);
 }
 

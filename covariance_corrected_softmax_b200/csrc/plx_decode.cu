@@ -139,7 +139,12 @@ __device__ void locate_range(const DecodeParams& p, int TK, RangeInfo* info, lon
 // ---------------------------------------------------------------------------
 // Main decode kernel.
 // ---------------------------------------------------------------------------
-template <typename T, int D, int HPW, bool PAGED>
+// MODE: kDecContiguous, kDecPaged (block-table loads), kDecState (contiguous
+// loads, softmax states written instead of the output).  Each is a separate
+// instance, so the common one carries no code of the others.
+constexpr int kDecContiguous = 0, kDecPaged = 1, kDecState = 2;
+
+template <typename T, int D, int HPW, int MODE>
 __global__ void __launch_bounds__(kDecThreads, 1)
     plx_decode_splitk_kernel(const __grid_constant__ CUtensorMap kmap,
                              const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
@@ -184,11 +189,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   grid_dep_launch_dependents();
   if (blockIdx.x == 0 && tid == 0) reinterpret_cast<long long*>(p.ws)[0] = info->total;
 
-  // Batches with an empty context produce zeros (out = 0 for an empty key set).
+  // Batches with an empty context produce zeros (out = 0 for an empty key set),
+  // or the empty state (m = -inf, everything else 0).
   for (int b = blockIdx.x; b < p.B; b += p.grid) {
     if (clamp_len(p.seqlens[b], p.S_max) == 0) {
-      for (int e = tid; e < p.Hq * D; e += blockDim.x)
-        store_elem<T>(p.out, (size_t)b * p.Hq * D + e, 0.f);
+      if constexpr (MODE == kDecState) {
+        for (int e = tid; e < p.Hq * PHF; e += blockDim.x)
+          p.state[(size_t)b * p.Hq * PHF + e] = (e % PHF == 0) ? -INFINITY : 0.f;
+      } else {
+        for (int e = tid; e < p.Hq * D; e += blockDim.x)
+          store_elem<T>(p.out, (size_t)b * p.Hq * D + e, 0.f);
+      }
     }
   }
 
@@ -197,7 +208,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   if (warp == kDecConsumerWarps) {
     // ------------------------------------------------------------ producer
-    if constexpr (!PAGED) {
+    if constexpr (MODE != kDecPaged) {
       // contiguous cache: one lane issues one K and one V load per tile
       if (lane == 0 && t0 < t1) {
         tma_prefetch_desc(&kmap);
@@ -561,7 +572,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             O += wt * src[4 + c];
             U += wt * src[4 + D + c];
           }
-          if (complete) {
+          if (MODE == kDecState && complete) {
+            float* sr = p.state + ((size_t)mt.b * p.Hq + h0 + g) * PHF;
+            if (c == 0) {
+              sr[0] = M;
+              sr[1] = L;
+              sr[2] = Z;
+              sr[3] = 0.f;
+            }
+            sr[4 + c] = O;
+            sr[4 + D + c] = U;
+          } else if (complete) {
             // out = (1 + tbar) o - u with tbar = Z/L, o = O/L, u = U/L
             const float inv = 1.f / L;
             const float val = ((1.f + Z * inv) * O - U) * inv;
@@ -655,10 +676,70 @@ __global__ void __launch_bounds__(256)
       record_error(p.err, kDevBadArgument);
       continue;
     }
+    if (p.state) {
+      float* sr = p.state + ((size_t)b * p.Hq + h0 + g) * PHF;
+      if (c == 0) {
+        sr[0] = M;
+        sr[1] = L;
+        sr[2] = Z;
+        sr[3] = 0.f;
+      }
+      sr[4 + c] = O;
+      sr[4 + D + c] = U;
+      continue;
+    }
     const float inv = 1.f / L;
     const float val = ((1.f + Z * inv) * O - U) * inv;
     store_elem<T>(p.out, ((size_t)b * p.Hq + h0 + g) * D + c, val);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of R softmax states per (b, h) row (R slices of one key set, e.g. the
+// context split over ranks) with the log-sum-exp rule, then
+// out = ((1 + z/l) o - u) / l (0 for an empty key set).  One block per row,
+// one thread per element.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(D)
+    plx_merge_states_kernel(const float* states, int R, long long rows, void* out) {
+  constexpr int PHF = part_head_floats<D>();
+  const int c = threadIdx.x;
+  for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
+    float M = -INFINITY;
+    for (int r = 0; r < R; ++r) M = fmaxf(M, states[((size_t)r * rows + row) * PHF]);
+    float L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
+    for (int r = 0; r < R; ++r) {
+      const float* sr = states + ((size_t)r * rows + row) * PHF;
+      const float w = merge_weight(sr[0], M);
+      L += w * sr[1];
+      Z += w * sr[2];
+      O += w * sr[4 + c];
+      U += w * sr[4 + D + c];
+    }
+    float val = 0.f;
+    if (L > 0.f) {
+      const float inv = 1.f / L;
+      val = ((1.f + Z * inv) * O - U) * inv;
+    }
+    store_elem<T>(out, (size_t)row * D + c, val);
+  }
+}
+
+cudaError_t launch_merge_states(const float* states, int R, long long rows, void* out, int d,
+                                bool bf16, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)(rows < 4096 ? rows : 4096);
+  if (d == 128) {
+    if (bf16) plx_merge_states_kernel<__nv_bfloat16, 128><<<grid, 128, 0, stream>>>(states, R, rows, out);
+    else plx_merge_states_kernel<float, 128><<<grid, 128, 0, stream>>>(states, R, rows, out);
+  } else if (d == 64) {
+    if (bf16) plx_merge_states_kernel<__nv_bfloat16, 64><<<grid, 64, 0, stream>>>(states, R, rows, out);
+    else plx_merge_states_kernel<float, 64><<<grid, 64, 0, stream>>>(states, R, rows, out);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -677,8 +758,9 @@ template <typename T, int D, int HPW>
 cudaError_t launch_decode_t(const CUtensorMap& kmap, const CUtensorMap& vmap,
                             const DecodeParams& p, cudaStream_t stream) {
   const int smem = decode_smem_bytes<T, D>(HPW);
-  auto kern = p.block_table ? plx_decode_splitk_kernel<T, D, HPW, true>
-                            : plx_decode_splitk_kernel<T, D, HPW, false>;
+  auto kern = p.block_table ? plx_decode_splitk_kernel<T, D, HPW, kDecPaged>
+               : p.state     ? plx_decode_splitk_kernel<T, D, HPW, kDecState>
+                             : plx_decode_splitk_kernel<T, D, HPW, kDecContiguous>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<p.grid, kDecThreads, smem, stream>>>(kmap, vmap, p);

@@ -87,6 +87,10 @@ struct DecodeParams {
   // j % page_size of page block_table[b * max_pages + j / page_size].
   const int32_t* block_table;
   int num_pages, page_size, max_pages;
+  // State mode (state != nullptr): instead of out, each (b, h) row's softmax
+  // state over this cache -- m (log2 units of the scaled scores), l, z, 0,
+  // o[D], u[D], unnormalised -- is written to state[(b * Hq + h) * (2D + 4)].
+  float* state;
 };
 
 // Tile metadata written by the producer next to each stage.

@@ -45,6 +45,9 @@ cudaError_t launch_prefill_tc(const PrefillTcArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(bool bf16, int d, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const DecodeParams& p, int hpw, cudaStream_t stream);
 int decode_tile_keys(bool bf16, int d);
+// out[row] from R softmax states [R, rows, 2d + 4] (see DecodeParams::state).
+cudaError_t launch_merge_states(const float* states, int R, long long rows, void* out, int d,
+                                bool bf16, cudaStream_t stream);
 // Writes the new token's K and V rows ([B, Hkv, d], elem_bytes per element) at
 // cache position seqlens[b] - 1 of every batch with a non-zero length.
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,

@@ -56,6 +56,10 @@ def lib() -> ctypes.CDLL:
         L.plx_decode_paged.restype = i
         L.plx_prefill_varlen.argtypes = [vp] * 7 + [i] * 9 + [f, vp]
         L.plx_prefill_varlen.restype = i
+        L.plx_decode_state.argtypes = [vp] * 6 + [i] * 6 + [f, vp, sz, vp]
+        L.plx_decode_state.restype = i
+        L.plx_merge_states.argtypes = [vp, i, vp, i, i, i, i, vp]
+        L.plx_merge_states.restype = i
         L.plx_status_string.argtypes = [i]
         L.plx_status_string.restype = ctypes.c_char_p
         L.plx_last_cuda_error.argtypes = []
@@ -199,6 +203,63 @@ def decode(q: torch.Tensor, rho: torch.Tensor, k_cache: torch.Tensor, v_cache: t
                           _stream(stream))
     _check(st, "plx_decode")
     return out
+
+
+def decode_state(q: torch.Tensor, rho: torch.Tensor, k_cache: torch.Tensor,
+                 v_cache: torch.Tensor, seqlens: torch.Tensor,
+                 softmax_scale: Optional[float] = None, state: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """decode() over this cache, returning each row's softmax state
+    [B, Hq, 2d + 4] fp32 (m, l, z, 0, o, u) instead of the output."""
+    _same(q, rho, k_cache, v_cache)
+    B, Hq, d = q.shape
+    S_max, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if rho.shape != q.shape or k_cache.shape != (B, S_max, Hkv, d) or \
+            v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch among q, rho, k_cache, v_cache")
+    if seqlens.dtype != torch.int32 or seqlens.device != q.device or seqlens.numel() != B:
+        raise ValueError("seqlens must be int32 [B] on the same device")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    if state is None:
+        state = torch.empty((B, Hq, 2 * d + 4), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, Hkv, d, S_max, device=q.device)
+    st = lib().plx_decode_state(_ptr(q), _ptr(rho), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+                                _ptr(state), B, Hq, Hkv, d, S_max, _dtype_code(q), scale,
+                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream))
+    _check(st, "plx_decode_state")
+    return state
+
+
+def merge_states(states: torch.Tensor, out_dtype: torch.dtype = torch.bfloat16,
+                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out [B, Hq, d] from states [R, B, Hq, 2d + 4] (decode_state layout)."""
+    if states.dtype != torch.float32 or states.dim() != 4 or not states.is_contiguous():
+        raise ValueError("states must be a contiguous fp32 [R, B, Hq, 2d + 4] tensor")
+    R, B, Hq, w = states.shape
+    d = (w - 4) // 2
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=out_dtype, device=states.device)
+    st = lib().plx_merge_states(_ptr(states), R, _ptr(out), B, Hq, d, _dtype_code(out),
+                                _stream(stream))
+    _check(st, "plx_merge_states")
+    return out
+
+
+def context_parallel_decode(q: torch.Tensor, rho: torch.Tensor, k_local: torch.Tensor,
+                            v_local: torch.Tensor, seqlens_local: torch.Tensor,
+                            softmax_scale: Optional[float] = None, group=None) -> torch.Tensor:
+    """Decode with the context split over the ranks of a torch.distributed group:
+    each rank holds a contiguous slice of every sequence's cache (seqlens_local =
+    the slice's filled length); the ranks' states are all-gathered (the one
+    exchange) and merged.  Every rank returns the full output."""
+    import torch.distributed as dist
+    state = decode_state(q, rho, k_local, v_local, seqlens_local, softmax_scale)
+    world = dist.get_world_size(group)
+    states = torch.empty((world,) + tuple(state.shape), dtype=state.dtype, device=state.device)
+    dist.all_gather_into_tensor(states, state, group=group)
+    return merge_states(states, out_dtype=q.dtype)
 
 
 def decode_paged(q: torch.Tensor, rho: torch.Tensor, k_pages: torch.Tensor,

@@ -149,6 +149,39 @@ PLX_API plx_status plx_decode(const void* q, const void* rho, const void* k_cach
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * plx_decode_state -- plx_decode, but instead of out it writes each (b, h)
+ * row's softmax state over this cache, so that a key set split into slices
+ * (for example a context spread over several GPUs) can be decoded slice by
+ * slice and merged with plx_merge_states.
+ *
+ *   state : [B, H_q, 2d + 4] fp32, device, 16-byte aligned, written; per row
+ *           m, l, z, 0, o[d], u[d]: m is the maximum of the scaled scores in
+ *           log2 units (softmax_scale * log2(e) * q.k), l = sum 2^(s - m),
+ *           z = sum 2^(s - m) (rho.k), o = sum 2^(s - m) v, u = sum 2^(s - m)
+ *           (rho.k) v (unnormalised); an empty key set gives m = -inf and
+ *           zeros
+ * Every other argument as plx_decode (out is not written).
+ */
+PLX_API plx_status plx_decode_state(const void* q, const void* rho, const void* k_cache,
+                                    const void* v_cache, const int32_t* seqlens, float* state,
+                                    int B, int H_q, int H_kv, int d, int S_max, plx_dtype dtype,
+                                    float softmax_scale, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/*
+ * plx_merge_states -- out = ((1 + Z/L) O - U) / L from R states of the same
+ * rows (log-sum-exp merge: M = max m_r, weights 2^(m_r - M); L, Z, O, U the
+ * weighted sums), the one exchange a context split over R slices needs
+ * (page 1 section 1.3 operator; the merge is exact up to rounding).
+ *
+ *   states : [R, B, H_q, 2d + 4] fp32 (plx_decode_state layout), device
+ *   out    : [B, H_q, d] in out_dtype (PLX_F32 or PLX_BF16), written; rows
+ *            whose R slices are all empty get 0
+ */
+PLX_API plx_status plx_merge_states(const float* states, int R, void* out, int B, int H_q, int d,
+                                    plx_dtype out_dtype, void* stream);
+
+/*
  * plx_decode_paged -- plx_decode over a paged KV cache (page 3: decoding keeps
  * a KV cache; a serving system stores it in fixed-size pages).
  *

@@ -158,6 +158,22 @@ def test_prefill_varlen_fp32_unsupported_and_empty_noop():
     assert _prefill_varlen(T=0, q=None) == plx.PLX_OK
 
 
+def test_decode_state_and_merge_reject_bad_arguments():
+    L = plx.lib()
+    # plx_decode_state: no state buffer, misaligned state
+    assert L.plx_decode_state(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 4, 2, 128, 64,
+                              plx.PLX_BF16, 1.0, FAKE, 1 << 20, None) == INV
+    assert L.plx_decode_state(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, 2, 4, 2, 128, 64,
+                              plx.PLX_BF16, 1.0, FAKE, 1 << 20, None) == INV
+    # plx_merge_states: R < 1, bad d, bad dtype, null pointers; B = 0 is a no-op
+    assert L.plx_merge_states(FAKE, 0, FAKE, 2, 4, 128, plx.PLX_BF16, None) == INV
+    assert L.plx_merge_states(FAKE, 2, FAKE, 2, 4, 96, plx.PLX_BF16, None) == INV
+    assert L.plx_merge_states(FAKE, 2, FAKE, 2, 4, 128, 9, None) == INV
+    assert L.plx_merge_states(None, 2, FAKE, 2, 4, 128, plx.PLX_F32, None) == INV
+    assert L.plx_merge_states(FAKE, 2, FAKE + 4, 2, 4, 128, plx.PLX_F32, None) == INV
+    assert L.plx_merge_states(None, 2, None, 0, 4, 128, plx.PLX_F32, None) == plx.PLX_OK
+
+
 def test_prefill_empty_is_noop():
     assert _prefill(B=0, q=None) == plx.PLX_OK
     assert _prefill(L=0, q=None) == plx.PLX_OK
