@@ -22,6 +22,13 @@
  *     LLA's solved probe Sigma^-1 mu does (page 1, 1.2-1.3);
  *   - the sign is the printed minus.
  *
+ * Pins: every routine here is checked against what the pages and the
+ * mathematics fix (textbook softmax attention at rho = 0, numpy's weighted
+ * covariance, LLA's weighted least-squares intercept, closed forms for one and
+ * two keys, uniform weights, invariances, hand-derived worked examples; see
+ * the tests).  Parity unpinned: the size of the correction for a trained W_R
+ * (the pages print no worked example or reference values for it).
+ *
  * Two forms are provided:
  *   PLXO_FORM_EXPLICIT  forms the d_k x d_v covariance matrix per row, then
  *                       contracts it with rho (the definition, written out);
