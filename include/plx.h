@@ -24,8 +24,10 @@
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers, owned by the caller, contiguous,
  *     row-major in the layouts given below, and 16-byte aligned.  The library
- *     never allocates, frees or synchronises; it only enqueues work.
- *   - dtype applies to q, rho, k, v and out alike.  Accumulation is fp32.
+ *     never allocates or frees, and only the diagnostic plx_device_error
+ *     synchronises; every other call only enqueues work.
+ *   - dtype applies to q, rho, k, v and out alike, unless an entry point takes
+ *     an out_dtype or writes fp32 states.  Accumulation is fp32.
  *     PLX_BF16 runs on the tensor cores (prefill) or streams a bf16 cache
  *     (decode); PLX_F32 computes every product in fp32 on the CUDA cores.
  *   - d (head dimension, d_k = d_v) must be 64 or 128; H_q must be a multiple
