@@ -87,3 +87,19 @@ def test_reference_arm_other_ranks_exit_quietly(monkeypatch, capsys):
         steps, warmup, gpus = 3, 3, 2
     assert bench.reference_arm(Args()) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_recorded_traffic_follows_the_source_digest(tmp_path, monkeypatch):
+    """bench.py reports DRAM traffic only for the kernel sources it was measured on."""
+    csrc = tmp_path / "covariance_corrected_softmax_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "a.cu").write_text("kernel v1\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    d1 = bench.source_digest(["a.cu"])
+    (tmp_path / "profiles" / "dram_traffic.txt").write_text(
+        "# header\nk1  w1  12345  %s  capture\n" % d1)
+    assert bench.recorded_traffic("k1", "w1", ["a.cu"]) == 12345.0
+    assert bench.recorded_traffic("k1", "other", ["a.cu"]) is None
+    (csrc / "a.cu").write_text("kernel v2\n")  # the kernel changed since the capture
+    assert bench.recorded_traffic("k1", "w1", ["a.cu"]) is None
