@@ -6,7 +6,11 @@ H_kv=8, d=128, context 4096 (``decode_b32_ctx4096``).  One step is one
 ``plx_decode`` call (score, probe score, online softmax, both accumulators,
 split merge).  The causal prefill rows of the hot path are measured in the same
 run on ``prefill_b8_l4096`` (B=8, L=4096, H_q=16, H_kv=8, d=128) and reported
-under ``"prefill"``.
+under ``"prefill"``, the long-context prefill ``prefill_b1_l32768`` (B=1,
+L=32768, H_q=32, H_kv=8) under ``"prefill_long"``, and the decode grid (batch
+1-2048 x context 128-32768, ragged lengths) under ``"sweep"``: per cell the
+device time per call with L2 flushed before every call, HBM GB/s from the
+actual lengths and the fraction of the measured copy bandwidth.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
 a device synchronisation, timed with CUDA events on the launching stream; the
@@ -42,6 +46,7 @@ if ROOT not in sys.path:
 METRIC = "decode tokens/s & HBM GB/s (% of roofline); prefill TFLOP/s (% bf16 peak)"
 HEADLINE = "decode_b32_ctx4096"
 PREFILL = "prefill_b8_l4096"
+PREFILL_LONG = "prefill_b1_l32768"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DECODE_SOURCES = ["plx_decode.cu", "plx_decode.cuh", "plx_device.cuh"]
 PREFILL_SOURCES = ["plx_prefill_tc.cu", "plx_device.cuh"]
@@ -334,6 +339,73 @@ def bench_prefill(plx, W, shape, steps, warmup, world, device, rank):
     return {"ms": ms, "clocks": clk.summary()}
 
 
+# ------------------------------------------------------------------ decode grid
+def bench_decode_sweep(plx, W, peaks, device, max_cells=None):
+    """Every cell of the decode grid (batch x context, ragged lengths U[ctx/2,
+    ctx], caches capped under 120e9 bytes).  Each call is timed alone with CUDA
+    events, after a 256 MiB buffer (twice the L2) has been written, so every
+    call reads its cache from HBM; the median over the calls is reported."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    cells = []
+    for cell in W.sweep_cells()[:max_cells]:
+        inp = W.make_decode(cell, seed=0, device=device)
+        ws = plx.decode_workspace(cell.B, cell.Hq, cell.Hkv, cell.d, cell.S_max, device=device)
+        out = torch.empty_like(inp["q"])
+        alg = decode_alg_bytes(cell, inp["seqlens"])
+        n = 10 if alg > 4e9 else 30
+
+        def call():
+            plx.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["seqlens"],
+                       softmax_scale=1.0, out=out, workspace=ws, stream=stream)
+
+        for _ in range(3):
+            call()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        for s_, e_ in ev:
+            flush.fill_(1)
+            s_.record(stream)
+            call()
+            e_.record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.median(s_.elapsed_time(e_) for s_, e_ in ev)
+        gbs = alg / (ms / 1e3) / 1e9
+        roof_us = alg / (peaks["hbm_gbs"] * 1e9) * 1e6
+        cells.append({"B": cell.B, "context": cell.ctx, "mean_len": float(inp["seqlens"].float().mean()),
+                      "us_per_call": ms * 1e3, "tokens_per_s": cell.B / (ms / 1e3),
+                      "hbm_gbs": gbs, "frac": gbs / peaks["hbm_gbs"], "bytes_per_call": alg,
+                      "calls": n, "launch_bound": roof_us < 20.0})
+        del inp, ws, out
+        torch.cuda.empty_cache()
+    assert plx.device_error() == 0, "decode kernels reported a device error in the sweep"
+    del flush
+    torch.cuda.empty_cache()
+    return cells
+
+
+def prefill_record(name, pshape, pr, psteps, world, peaks, peak_src, traffic):
+    pms = pr["ms"] / psteps
+    tflops = pshape.flops() / (pms / 1e3) / 1e12
+    return {
+        "workload": name, "B": pshape.B, "L": pshape.L, "H_q": pshape.Hq,
+        "H_kv": pshape.Hkv, "d": pshape.d, "causal": pshape.causal, "steps": psteps,
+        "ms_per_call": pms, "tflops": tflops,
+        "tokens_per_s": aggregate_rate(world, pshape.B * pshape.L, psteps, pr["ms"]),
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     # the leg runs `psteps` calls back to back (a long loop under
+                     # the power cap): the sustained GEMM figure, for comparison
+                     "peak_sustained": peaks["bf16_tflops_sustained"],
+                     "frac_sustained": tflops / peaks["bf16_tflops_sustained"],
+                     "flops_per_call": pshape.flops(), "traffic": traffic},
+        "gpu_launches_per_call": 1,
+        "clocks": pr["clocks"],
+    }
+
+
 # -------------------------------------------------------------------- reference
 def reference_arm(args):
     """The oracle as it stands on the host cores, same workload and metric."""
@@ -408,6 +480,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-I/O leg (profiling)")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the decode grid")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -442,35 +515,32 @@ def main():
                    "call": "plx_decode_append (KV append + decode)",
                    "gpu_launches": 3 * args.steps}
 
-    prefill = None
+    prefill = prefill_long = None
     if not args.no_prefill:
-        pshape = W.WORKLOADS[PREFILL]
-        psteps = max(3, min(200, args.steps // 10))
-        pr = bench_prefill(plx, W, pshape, psteps, max(3, min(args.warmup, 10)), world, device,
-                           rank)
-        if "ms" in pr:
-            pms = pr["ms"] / psteps
-            tflops = pshape.flops() / (pms / 1e3) / 1e12
-            prefill = {
-                "workload": PREFILL, "B": pshape.B, "L": pshape.L, "H_q": pshape.Hq,
-                "H_kv": pshape.Hkv, "d": pshape.d, "causal": pshape.causal, "steps": psteps,
-                "ms_per_call": pms, "tflops": tflops,
-                "tokens_per_s": aggregate_rate(world, pshape.B * pshape.L, psteps, pr["ms"]),
-                "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
-                             "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
-                             "peak_source": f"{peak_src} bf16 dense (burst)",
-                             # the leg runs `psteps` calls back to back (a long loop under
-                             # the power cap): the sustained GEMM figure, for comparison
-                             "peak_sustained": peaks["bf16_tflops_sustained"],
-                             "frac_sustained": tflops / peaks["bf16_tflops_sustained"],
-                             "flops_per_call": pshape.flops(),
-                             "traffic": recorded_traffic("plx_prefill_tc", PREFILL,
-                                                         PREFILL_SOURCES)},
-                "gpu_launches_per_call": 1,
-                "clocks": pr["clocks"],
-            }
-        else:
-            prefill = {"workload": PREFILL, **pr}
+        for name, psteps in ((PREFILL, 40), (PREFILL_LONG, 8)):
+            pshape = W.WORKLOADS[name]
+            pr = bench_prefill(plx, W, pshape, psteps, 3, world, device, rank)
+            if "ms" in pr:
+                rec_p = prefill_record(name, pshape, pr, psteps, world, peaks, peak_src,
+                                       recorded_traffic("plx_prefill_tc", name, PREFILL_SOURCES))
+            else:
+                rec_p = {"workload": name, **pr}
+            if name == PREFILL:
+                prefill = rec_p
+            else:
+                prefill_long = rec_p
+
+    sweep = None
+    if not args.no_sweep:
+        with ClockSampler(gpu_index()) as clk:
+            cells = bench_decode_sweep(plx, W, peaks, device)
+        long_ctx = [c for c in cells if c["context"] >= 8192 and not c["launch_bound"]]
+        sweep = {"grid": "H_q=16, H_kv=8, d=128, bf16; batch x context, lengths U[ctx/2, ctx]",
+                 "timing": "median of per-call CUDA-event times, 256 MiB L2 flush before each call",
+                 "peak": peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy bandwidth",
+                 "cells": cells,
+                 "min_frac_ctx_ge_8192": min((c["frac"] for c in long_ctx), default=None),
+                 "clocks": clk.summary()}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -493,6 +563,8 @@ def main():
         "gpu_launches": 2 * args.steps,
         "clocks": dec["clocks"],
         "prefill": prefill,
+        "prefill_long": prefill_long,
+        "sweep": sweep,
     }
     if rank == 0:
         print(json.dumps(rec), flush=True)

@@ -4,14 +4,16 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <mutex>
 
 #include "plx.h"
 #include "plx_launch.h"
 
 
-// The device error word (one per device context); kernels receive its address.
-__device__ unsigned plx_g_device_error = 0;
+// The device status block (one per device context): the error word, which
+// kernels receive the address of, and the limit of their bounded waits.
+__device__ plx::DeviceStatus plx_g_status = {0u, 0u, plx::kWaitLimitNs};
 
 namespace {
 
@@ -43,7 +45,7 @@ cudaError_t device_info(int* sms, unsigned** err) {
     e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, plx_g_device_error);
+    e = cudaGetSymbolAddress(&ptr, plx_g_status);
     if (e != cudaSuccess) return e;
     g_err_ptr[dev] = static_cast<unsigned*>(ptr);
     g_sm_count[dev] = n;
@@ -124,15 +126,37 @@ plx_status plx_device_error(int* code, int clear) {
   unsigned v = 0;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaMemcpyFromSymbol(&v, plx_g_device_error, sizeof(v));
+  e = cudaMemcpyFromSymbol(&v, plx_g_status, sizeof(v), offsetof(plx::DeviceStatus, error));
   if (e != cudaSuccess) return cuda_fail(e);
   if (clear) {
     unsigned z = 0;
-    e = cudaMemcpyToSymbol(plx_g_device_error, &z, sizeof(z));
+    e = cudaMemcpyToSymbol(plx_g_status, &z, sizeof(z), offsetof(plx::DeviceStatus, error));
     if (e != cudaSuccess) return cuda_fail(e);
   }
   *code = static_cast<int>(v);
   return PLX_OK;
+}
+
+plx_status plx_set_wait_limit_ns(unsigned long long ns) {
+  t_last_cuda_error = 0;
+  if (ns == 0) ns = plx::kWaitLimitNs;
+  if (ns < 1000ull || ns > 60000000000ull) return PLX_ERR_INVALID_ARGUMENT;
+  const unsigned long long v = ns;
+  cudaError_t e = cudaDeviceSynchronize();  // no kernel may be mid-wait
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemcpyToSymbol(plx_g_status, &v, sizeof(v), offsetof(plx::DeviceStatus, wait_limit_ns));
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaDeviceSynchronize();
+  return e == cudaSuccess ? PLX_OK : cuda_fail(e);
+}
+
+plx_status plx_selftest_wait(void* stream) {
+  t_last_cuda_error = 0;
+  unsigned* err = nullptr;
+  cudaError_t e = device_info(nullptr, &err);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = plx::launch_selftest_wait(err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PLX_OK : cuda_fail(e);
 }
 
 size_t plx_decode_workspace_bytes(int B, int H_q, int H_kv, int d, int S_max) {
@@ -364,8 +388,15 @@ plx_status plx_decode_append(const void* q, const void* rho, const void* k_new,
 
 plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k, const void* v,
                            void* out, float* lse, int causal, int B, int L, int H_q, int H_kv,
-                           int d, plx_dtype dtype, plx_dtype out_dtype, float softmax_scale,
-                           void* stream) {
+                           int d, plx_dtype dtype, float softmax_scale, void* stream) {
+  return plx_prefill_fwd_ex(q, rho, k, v, out, lse, causal, B, L, H_q, H_kv, d, dtype, dtype,
+                            softmax_scale, stream);
+}
+
+plx_status plx_prefill_fwd_ex(const void* q, const void* rho, const void* k, const void* v,
+                              void* out, float* lse, int causal, int B, int L, int H_q, int H_kv,
+                              int d, plx_dtype dtype, plx_dtype out_dtype, float softmax_scale,
+                              void* stream) {
   t_last_cuda_error = 0;
   if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
   if (out_dtype != dtype && !(dtype == PLX_BF16 && out_dtype == PLX_F32))

@@ -27,6 +27,19 @@ namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(1) << 20;  // 1 MiB
 
+// Workspace plx_decode needs on a device with `sms` multiprocessors: a header
+// plus two partial-state slots per CTA of the persistent grid (at most one CTA
+// per SM), each slot holding `hpw` heads' (m, l, z, pad, o[d], u[d]).
+constexpr size_t static_need(int sms, int d, int hpw) {
+  return (size_t)(plx::kWsHeaderFloats + (size_t)2 * sms * (plx::kPartHeader + hpw * (2 * d + 4))) *
+         sizeof(float);
+}
+// B200 (148 SMs) at the widest slot (d = 128, two heads per pass) fits, and so
+// does any device with up to 250 SMs.
+static_assert(static_need(148, 128, 2) <= kStaticScratchBytes, "B200 must fit");
+static_assert(static_need(250, 128, 2) <= kStaticScratchBytes, "250 SMs must fit");
+static_assert(static_need(251, 128, 2) > kStaticScratchBytes, "limit stated in plx.h");
+
 // The scratch itself.  In host code this name is only a stand-in for the
 // symbol, not a device address: kernels get the address from
 // cudaGetSymbolAddress below.

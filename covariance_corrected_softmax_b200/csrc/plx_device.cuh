@@ -21,8 +21,16 @@ enum DeviceError : unsigned {
   kDevNonFinite = 3,         // a result was not finite (inputs out of range)
 };
 
-// The word lives in the library (plx_abi.cu); kernels get its address as a
-// parameter.
+// The device status block lives in the library (plx_abi.cu), one per device;
+// kernels get the address of its first word (the error code) as a parameter.
+// The wall-clock limit of every bounded wait sits in the same block, so a
+// diagnostic entry point can shorten it without rebuilding the kernels.
+struct DeviceStatus {
+  unsigned error;                   // first DeviceError recorded (0 = none)
+  unsigned reserved;
+  unsigned long long wait_limit_ns; // limit of one bounded wait
+};
+
 __device__ __forceinline__ void record_error(unsigned* err, unsigned code) {
   if (err) atomicCAS(err, 0u, code);
 }
@@ -33,9 +41,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Wall-clock limit of a single wait (ns).  Long enough for any legitimate
-// stall (including profiler replay), short enough to give the GPU back.
+// Default wall-clock limit of a single wait (ns).  Long enough for any
+// legitimate stall (including profiler replay), short enough to give the GPU
+// back.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Backstop on the number of polls of one wait, should the wall clock stop: a
+// poll takes tens of nanoseconds or more, so this is tens of seconds.
+constexpr uint32_t kWaitMaxPolls = 1u << 30;
+
+// The wait limit in force on this device (the status block's, or the default
+// when a kernel runs without one).
+__device__ __forceinline__ uint64_t wait_limit_ns(const unsigned* err) {
+  if (!err) return kWaitLimitNs;
+  return reinterpret_cast<const volatile DeviceStatus*>(err)->wait_limit_ns;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -147,17 +166,20 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // Waits until the phase with the given parity has completed.  Returns false
-// (and records kDevTimeoutMbarrier) if the wall-clock limit runs out or if
-// *abort becomes nonzero (another role of the CTA gave up).
+// (and records kDevTimeoutMbarrier) if the wall-clock limit runs out (or the
+// poll backstop is reached) or if *abort becomes nonzero (another role of the
+// CTA gave up).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort, unsigned* err) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = globaltimer_ns();
+  uint64_t limit = 0;
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++spins & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (limit == 0) limit = wait_limit_ns(err);
+      if (globaltimer_ns() - t0 > limit || spins >= kWaitMaxPolls) {
         record_error(err, kDevTimeoutMbarrier);
         *abort = 1;
         return false;

@@ -54,6 +54,11 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache
                              const int32_t* seqlens, int B, int Hkv, int d, int elem_bytes,
                              int S_max, cudaStream_t stream);
 
+// One warp that waits on an mbarrier nothing ever completes, with the
+// device's bounded wait: it records kDevTimeoutMbarrier when the limit runs out
+// and returns (the failure-detection self-test).
+cudaError_t launch_selftest_wait(unsigned* err, cudaStream_t stream);
+
 // TMA descriptor encoder (cuTensorMapEncodeTiled through the runtime's driver
 // entry point); null if unavailable.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -44,8 +44,10 @@ def lib() -> ctypes.CDLL:
                 "`python -m covariance_corrected_softmax_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-        L.plx_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp]
+        L.plx_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp]
         L.plx_prefill_fwd.restype = i
+        L.plx_prefill_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp]
+        L.plx_prefill_fwd_ex.restype = i
         L.plx_decode_workspace_bytes.argtypes = [i, i, i, i, i]
         L.plx_decode_workspace_bytes.restype = sz
         L.plx_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, sz, vp]
@@ -66,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.plx_last_cuda_error.restype = i
         L.plx_device_error.argtypes = [ctypes.POINTER(i), i]
         L.plx_device_error.restype = i
+        L.plx_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.plx_set_wait_limit_ns.restype = i
+        L.plx_selftest_wait.argtypes = [vp]
+        L.plx_selftest_wait.restype = i
         L.plx_version.argtypes = []
         L.plx_version.restype = i
         _lib = L
@@ -127,10 +133,14 @@ def prefill(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch.Tensor
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
-    st = lib().plx_prefill_fwd(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out),
-                               _ptr(lse) if return_lse else None, int(bool(causal)), B, L, Hq,
-                               Hkv, d, _dtype_code(q), _dtype_code(out), scale, _stream(stream))
-    _check(st, "plx_prefill_fwd")
+    args = (_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out), _ptr(lse) if return_lse else None,
+            int(bool(causal)), B, L, Hq, Hkv, d, _dtype_code(q))
+    if out.dtype == q.dtype:
+        st, name = lib().plx_prefill_fwd(*args, scale, _stream(stream)), "plx_prefill_fwd"
+    else:
+        st = lib().plx_prefill_fwd_ex(*args, _dtype_code(out), scale, _stream(stream))
+        name = "plx_prefill_fwd_ex"
+    _check(st, name)
     return out, (lse if return_lse else None)
 
 
@@ -249,17 +259,27 @@ def merge_states(states: torch.Tensor, out_dtype: torch.dtype = torch.bfloat16,
 
 def context_parallel_decode(q: torch.Tensor, rho: torch.Tensor, k_local: torch.Tensor,
                             v_local: torch.Tensor, seqlens_local: torch.Tensor,
-                            softmax_scale: Optional[float] = None, group=None) -> torch.Tensor:
+                            softmax_scale: Optional[float] = None, group=None,
+                            out_dtype: Optional[torch.dtype] = None) -> torch.Tensor:
     """Decode with the context split over the ranks of a torch.distributed group:
     each rank holds a contiguous slice of every sequence's cache (seqlens_local =
     the slice's filled length); the ranks' states are all-gathered (the one
-    exchange) and merged.  Every rank returns the full output."""
+    exchange) and merged.  Every rank returns the full output (out_dtype, by
+    default q's).  NCCL groups gather device tensors; other backends (gloo)
+    gather through host memory."""
     import torch.distributed as dist
     state = decode_state(q, rho, k_local, v_local, seqlens_local, softmax_scale)
     world = dist.get_world_size(group)
-    states = torch.empty((world,) + tuple(state.shape), dtype=state.dtype, device=state.device)
-    dist.all_gather_into_tensor(states, state, group=group)
-    return merge_states(states, out_dtype=q.dtype)
+    if dist.get_backend(group) == "nccl":
+        states = torch.empty((world,) + tuple(state.shape), dtype=state.dtype,
+                             device=state.device)
+        dist.all_gather_into_tensor(states, state, group=group)
+    else:
+        host = state.cpu()
+        parts = [torch.empty_like(host) for _ in range(world)]
+        dist.all_gather(parts, host, group=group)
+        states = torch.stack(parts).to(state.device)
+    return merge_states(states, out_dtype=out_dtype or q.dtype)
 
 
 def decode_paged(q: torch.Tensor, rho: torch.Tensor, k_pages: torch.Tensor,
@@ -328,3 +348,14 @@ def device_error(clear: bool = True) -> int:
     code = ctypes.c_int(0)
     _check(lib().plx_device_error(ctypes.byref(code), int(clear)), "plx_device_error")
     return code.value
+
+
+def set_wait_limit_ns(ns: int = 0) -> None:
+    """Diagnostic: the limit of every bounded wait in the kernels on the current
+    device (0 restores the default, 2 s); synchronises."""
+    _check(lib().plx_set_wait_limit_ns(int(ns)), "plx_set_wait_limit_ns")
+
+
+def selftest_wait(stream=None) -> None:
+    """Diagnostic: enqueue a kernel whose one bounded wait can only run out."""
+    _check(lib().plx_selftest_wait(_stream(stream)), "plx_selftest_wait")

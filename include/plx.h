@@ -75,27 +75,43 @@ typedef enum plx_dtype { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
  *
  *   q, rho : [B, L, H_q, d]   queries and probes (one probe per query row)
  *   k, v   : [B, L, H_kv, d]  keys and values
- *   out    : [B, L, H_q, d]   written, in out_dtype
+ *   out    : [B, L, H_q, d]   written, in dtype
  *   lse    : [B, H_q, L] fp32, written if non-NULL: natural-log
  *            log-sum-exp of the scaled scores of each row (the softmax
  *            normaliser; independent of rho)
  *   causal : 1 = row i sees keys 0..i; 0 = every row sees all L keys
- *   dtype  : of q, rho, k, v
- *   out_dtype : of out; equal to dtype, or PLX_F32 with bf16 inputs (an fp32
- *            result avoids the final rounding to bf16's 8 significant bits)
+ *   dtype  : of q, rho, k, v and out
  *   softmax_scale : the score scale (1/sqrt(d) in the textbook form,
  *            page 1 section 1.1); any finite value
  * Sizes: B, L, H_q, H_kv >= 1 (B == 0 or L == 0 is a no-op returning PLX_OK).
  * PLX_BF16 computes S = q.k and t = rho.k from the bf16 inputs on the tensor
- * cores and the two value products in fp16 x fp16 (fp32 accumulation), so
- * |v| and |rho . k| must stay below 65504; a non-finite result sets device
+ * cores and the two value products in fp16 x fp16 with fp32 accumulation: P
+ * and P t are rounded to fp16 (11 significant bits), V is scaled by a power of
+ * two per key tile and work unit (block floating point, undone in the
+ * epilogue) so that every finite bf16 V keeps 11 significant bits relative to
+ * the largest |v| of its tile.  A result that does not fit fp32 sets device
  * error 3 (plx_device_error).
  * Operator definition: page 1 section 1.3 and page 3 (see the file header).
  */
 PLX_API plx_status plx_prefill_fwd(const void* q, const void* rho, const void* k,
                                    const void* v, void* out, float* lse, int causal, int B,
                                    int L, int H_q, int H_kv, int d, plx_dtype dtype,
-                                   plx_dtype out_dtype, float softmax_scale, void* stream);
+                                   float softmax_scale, void* stream);
+
+/*
+ * plx_prefill_fwd_ex -- plx_prefill_fwd with the output dtype chosen apart
+ * from the input dtype.
+ *
+ *   out_dtype : dtype of out; equal to dtype, or PLX_F32 with PLX_BF16 inputs
+ *               (the fp32 result before the final rounding to bf16's 8
+ *               significant bits)
+ * Every other argument, requirement and error as plx_prefill_fwd.  With
+ * out_dtype == dtype the call is plx_prefill_fwd.
+ */
+PLX_API plx_status plx_prefill_fwd_ex(const void* q, const void* rho, const void* k,
+                                      const void* v, void* out, float* lse, int causal, int B,
+                                      int L, int H_q, int H_kv, int d, plx_dtype dtype,
+                                      plx_dtype out_dtype, float softmax_scale, void* stream);
 
 /*
  * plx_prefill_varlen -- plx_prefill_fwd over sequences of different lengths
@@ -244,9 +260,13 @@ PLX_API plx_status plx_decode_append(const void* q, const void* rho, const void*
  * Arguments and results are those of plx_decode without the workspace: the
  * caller still passes every input and the output.  The workspace is a fixed
  * 1 MiB array in the library's device memory, present on every GPU that loads
- * the library until the process exits.  A shape whose workspace would exceed
- * 1 MiB returns PLX_ERR_WORKSPACE_TOO_SMALL (B200's 148 SMs need about 0.6 MiB
- * for d = 128, so every valid shape fits there).  No allocation of any kind.
+ * the library until the process exits.  The workspace a shape needs is
+ * plx_decode_workspace_bytes(...) = 64 + 8 * SMs * (4 + h * (2 d + 4)) bytes,
+ * with SMs the device's multiprocessor count and h = 2 if H_q / H_kv is even,
+ * else 1; a shape needing more than 1 MiB returns PLX_ERR_WORKSPACE_TOO_SMALL.
+ * At d = 128, h = 2 that is 4192 bytes per SM: B200's 148 SMs need 0.59 MiB,
+ * and every valid shape fits on any device with up to 250 SMs.  No allocation
+ * of any kind.
  *
  * The first call on a device looks up the array's device address with
  * cudaGetSymbolAddress (once per device, with that device current); make that
@@ -274,6 +294,27 @@ PLX_API int plx_last_cuda_error(void);
  * Returns PLX_OK or PLX_ERR_CUDA.
  */
 PLX_API plx_status plx_device_error(int* code, int clear);
+
+/*
+ * plx_set_wait_limit_ns -- diagnostic: the wall-clock limit of every bounded
+ * wait in the library's kernels on the current device (default 2 s; ns = 0
+ * restores it; otherwise 1000 <= ns <= 6e10).  Meant for tests of the failure
+ * detection: a shorter limit makes a stalled wait give up sooner, and a limit
+ * shorter than a legitimate stall makes a correct kernel give up and report a
+ * timeout.  Synchronises the device.  The pages have no counterpart to this
+ * entry point.
+ */
+PLX_API plx_status plx_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * plx_selftest_wait -- diagnostic: enqueues on stream one warp that waits on a
+ * barrier nothing ever completes, through the same bounded wait every kernel of
+ * the library uses.  When the limit (plx_set_wait_limit_ns) runs out the kernel
+ * records code 1 in the device error word (plx_device_error) and returns; the
+ * context stays usable.  Returns PLX_OK once enqueued.  The pages have no
+ * counterpart to this entry point.
+ */
+PLX_API plx_status plx_selftest_wait(void* stream);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 PLX_API int plx_version(void);

@@ -49,13 +49,41 @@ def _decode(**kw):
 
 
 def _prefill(**kw):
+    """plx_prefill_fwd, or plx_prefill_fwd_ex when out_dtype is given."""
     a = dict(q=FAKE, rho=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=None, causal=1, B=1, L=16, Hq=2,
              Hkv=1, d=64, dtype=plx.PLX_F32, out_dtype=None, scale=0.125)
     a.update(kw)
-    od = a["dtype"] if a["out_dtype"] is None else a["out_dtype"]
-    return plx.lib().plx_prefill_fwd(a["q"], a["rho"], a["k"], a["v"], a["out"], a["lse"],
-                                     a["causal"], a["B"], a["L"], a["Hq"], a["Hkv"], a["d"],
-                                     a["dtype"], od, a["scale"], None)
+    head = (a["q"], a["rho"], a["k"], a["v"], a["out"], a["lse"], a["causal"], a["B"], a["L"],
+            a["Hq"], a["Hkv"], a["d"], a["dtype"])
+    if a["out_dtype"] is None:
+        return plx.lib().plx_prefill_fwd(*head, a["scale"], None)
+    return plx.lib().plx_prefill_fwd_ex(*head, a["out_dtype"], a["scale"], None)
+
+
+def _prototype(name):
+    """Parameter list of a declaration in plx.h, whitespace-normalised."""
+    with open(HEADER) as f:
+        text = f.read()
+    m = re.search(r"PLX_API\s+plx_status\s+" + name + r"\s*\(([^;]*)\)\s*;", text)
+    assert m, name
+    return [" ".join(p.split()) for p in m.group(1).split(",")]
+
+
+def test_prefill_fwd_prototype_is_the_specified_one():
+    """plx_prefill_fwd(q, rho, k, v, out, lse, causal, B, L, H_q, H_kv, d, dtype,
+    softmax_scale, stream): one dtype for q, rho, k, v and out."""
+    assert _prototype("plx_prefill_fwd") == [
+        "const void* q", "const void* rho", "const void* k", "const void* v", "void* out",
+        "float* lse", "int causal", "int B", "int L", "int H_q", "int H_kv", "int d",
+        "plx_dtype dtype", "float softmax_scale", "void* stream"]
+    ex = _prototype("plx_prefill_fwd_ex")
+    assert ex[:13] == _prototype("plx_prefill_fwd")[:13]
+    assert ex[13:] == ["plx_dtype out_dtype", "float softmax_scale", "void* stream"]
+    assert _prototype("plx_decode") == [
+        "const void* q", "const void* rho", "const void* k_cache", "const void* v_cache",
+        "const int32_t* seqlens", "void* out", "int B", "int H_q", "int H_kv", "int d",
+        "int S_max", "plx_dtype dtype", "float softmax_scale", "void* workspace",
+        "size_t workspace_bytes", "void* stream"]
 
 
 INV = plx.PLX_ERR_INVALID_ARGUMENT
@@ -128,6 +156,7 @@ def test_decode_append_empty_batch_is_noop():
     dict(d=32), dict(Hq=2, Hkv=3), dict(causal=2), dict(L=-1), dict(dtype=3),
     dict(scale=float("nan")), dict(q=None), dict(rho=None), dict(out=None), dict(k=FAKE + 8),
     dict(lse=FAKE + 2), dict(out_dtype=plx.PLX_BF16), dict(out_dtype=5),
+    dict(dtype=plx.PLX_BF16, scale=float("inf")), dict(dtype=plx.PLX_BF16, out_dtype=7),
 ])
 def test_prefill_rejects(kw):
     assert _prefill(**kw) == INV
@@ -177,6 +206,7 @@ def test_decode_state_and_merge_reject_bad_arguments():
 def test_prefill_empty_is_noop():
     assert _prefill(B=0, q=None) == plx.PLX_OK
     assert _prefill(L=0, q=None) == plx.PLX_OK
+    assert _prefill(B=0, q=None, dtype=plx.PLX_BF16, out_dtype=plx.PLX_F32) == plx.PLX_OK
 
 
 def test_workspace_query_rejects_bad_shapes():
@@ -195,3 +225,10 @@ def test_product_path_does_not_import_oracle():
                     src = f.read()
                 assert "import oracle" not in src and "from oracle" not in src, fn
                 assert "plx_oracle" not in src and "plxo_" not in src, fn
+
+
+def test_wait_limit_rejects_out_of_range_values():
+    # checked before any device call
+    L = plx.lib()
+    assert L.plx_set_wait_limit_ns(999) == INV
+    assert L.plx_set_wait_limit_ns(61 * 10 ** 9) == INV

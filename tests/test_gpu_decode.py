@@ -77,6 +77,36 @@ def test_decode_small_shapes(case):
               output_rounding=True)
 
 
+@pytest.mark.parametrize("case", [c for c in SMALL if c[-1] == torch.bfloat16],
+                         ids=[f"c{i}" for i, c in enumerate(SMALL) if c[-1] == torch.bfloat16])
+def test_decode_small_shapes_fp32_result_strict_bar(case):
+    """The bf16 edge shapes above at the plain 2e-2 RMS bar, with no allowance
+    for the output format: the result is taken in fp32 through the state path
+    (plx_decode_state, then plx_merge_states of the single slice into fp32),
+    which runs the same main kernel and merge arithmetic as plx_decode."""
+    B, Hq, Hkv, d, S, lens, dt = case
+    g = torch.Generator(device=DEV).manual_seed(7 + B * 31 + S)
+    s = d ** -0.25
+    q = (torch.randn(B, Hq, d, generator=g, device=DEV) * s).to(dt)
+    rho = (torch.randn(B, Hq, d, generator=g, device=DEV) * 0.3).to(dt)
+    k = (torch.randn(B, S, Hkv, d, generator=g, device=DEV) * s).to(dt)
+    v = (torch.randn(B, S, Hkv, d, generator=g, device=DEV) * s).to(dt)
+    if lens is None:
+        sl = torch.randint(0, S + 1, (B,), generator=g, device=DEV, dtype=torch.int32)
+    else:
+        sl = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    scale = 1.0 / np.sqrt(d)
+    st = plx.decode_state(q, rho, k, v, sl, softmax_scale=scale)
+    out = plx.merge_states(st[None].contiguous(), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref, _ = oracle.decode(q, rho, k, v, sl, scale)
+    check_out(to_np(out), ref, bf16=True, what=f"fp32 result {case[:5]}")
+    # and plx_decode's bf16 output is that fp32 result rounded once
+    bf = plx.decode(q, rho, k, v, sl, softmax_scale=scale)
+    torch.cuda.synchronize()
+    assert torch.equal(bf, out.to(torch.bfloat16))
+
+
 @pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
 def test_decode_ignores_rows_beyond_seqlen(dt):
     """Cache rows past seqlens[b] (here NaN and inf) never reach the output."""

@@ -2,8 +2,11 @@
 allocate device memory (a per-token serving loop that must stay out of the
 allocator, a plugin whose host owns the device memory pool, a C caller with no
 device allocator).  It runs the plx_decode kernels with a fixed workspace
-array inside the library, so its output must equal plx_decode's, call after
-call, while the shared array carries state from one call to the next.
+array inside the library, so its output must equal plx_decode's bit for bit,
+call after call, while the shared array carries state from one call to the
+next: a full-grid call first, then calls whose grids are smaller (their CTAs
+must not read slots that the earlier, larger grid left behind), with ragged
+lengths, an fp32 cache and d = 64.
 
 This file is collected last on purpose: it must pass both on its own in a
 fresh process (where its first call does the per-device set-up) and after
@@ -39,14 +42,39 @@ def static_decode(inp, scale):
     return st, out
 
 
-def test_static_workspace_decode_matches_plx_decode_two_calls():
-    first = W.make_decode(W.WORKLOADS["decode_b32_ctx4096"], seed=0, device=DEV)
-    second = W.make_decode(W.DecodeShape(B=5, Hq=16, Hkv=8, d=128, S_max=777, ctx=777,
-                                         ragged=True), seed=3, device=DEV)
-    for n, inp in enumerate((first, second)):
+def _small(B, Hq, Hkv, d, S, lens, dt, seed):
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    s = d ** -0.25
+    return dict(q=(torch.randn(B, Hq, d, generator=g, device=DEV) * s).to(dt),
+                rho=(torch.randn(B, Hq, d, generator=g, device=DEV) * 0.3).to(dt),
+                k_cache=(torch.randn(B, S, Hkv, d, generator=g, device=DEV) * s).to(dt),
+                v_cache=(torch.randn(B, S, Hkv, d, generator=g, device=DEV) * s).to(dt),
+                seqlens=torch.tensor(lens, dtype=torch.int32, device=DEV))
+
+
+def test_static_workspace_decode_matches_plx_decode_call_after_call():
+    calls = [
+        ("decode_b32_ctx4096 (full grid)",
+         W.make_decode(W.WORKLOADS["decode_b32_ctx4096"], seed=0, device=DEV)),
+        ("B=5 ragged, S_max=777 (full grid)",
+         W.make_decode(W.DecodeShape(B=5, Hq=16, Hkv=8, d=128, S_max=777, ctx=777, ragged=True),
+                       seed=3, device=DEV)),
+        ("B=1, H_q=2, H_kv=1, 64 keys (one tile, grid of 1)",
+         _small(1, 2, 1, 128, 64, [64], torch.bfloat16, seed=4)),
+        ("B=3 fp32, d=64, ragged (small grid)",
+         _small(3, 4, 2, 64, 150, [150, 0, 49], torch.float32, seed=5)),
+        ("B=2, 300 keys (a few tiles, split segments)",
+         _small(2, 16, 8, 128, 300, [300, 97], torch.bfloat16, seed=6)),
+    ]
+    for n, (what, inp) in enumerate(calls):
         ref = plx.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["seqlens"],
                          softmax_scale=1.0)
+        torch.cuda.synchronize()
         st, out = static_decode(inp, 1.0)
-        assert st == plx.PLX_OK, f"call {n}: {plx.status_string(st)}"
-        check_out(to_np(out), to_np(ref), bf16=True, what=f"static-workspace call {n}")
+        assert st == plx.PLX_OK, f"call {n} ({what}): {plx.status_string(st)}"
+        if not torch.equal(out, ref):
+            # say by how much before failing on the bit comparison
+            check_out(to_np(out), to_np(ref), bf16=out.dtype == torch.bfloat16,
+                      what=f"static-workspace call {n} ({what})")
+        assert torch.equal(out, ref), f"call {n} ({what}): not bit-identical to plx_decode"
     assert plx.device_error() == 0
