@@ -22,6 +22,12 @@ Operator (page 1 "Parallax: Parameterized Local Linear Attention Gives
 Transformers a 'Second Eye'", section 1.3; page 3 "Parallax keeps softmax, adds
 covariance correction branch"): ``out_i = o_SA,i - Sigma_KV^(i)^T rho_i`` with
 ``Sigma_KV^(i) = sum_j a_ij (k_j - mu_i)(v_j - o_SA,i)^T``.
+
+Also here: the probe projection ``rho = W_R x`` (page 1 section 1.3: one extra
+projection matrix; page 3: rho_i = W_R x_i), and the gradients of the prefill
+operator (the pages print none; the derivation is written out in
+``plx_oracle.c``), pinned by central finite differences of the forward and by
+fp64 autograd of the explicit-covariance definition.
 """
 from __future__ import annotations
 
@@ -73,6 +79,16 @@ class Oracle:
                       ctypes.c_int, dp, dp, ctypes.c_int]
         f.restype = ctypes.c_int
         self._rows = f
+        i64 = ctypes.c_int64
+        f = self._lib.plxo_probe
+        f.argtypes = [dp, dp, dp, i64, i64, i64]
+        f.restype = ctypes.c_int
+        self._probe = f
+        f = self._lib.plxo_prefill_bwd
+        f.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64, ctypes.c_int,
+                      ctypes.c_double, dp, dp, dp, dp, ctypes.c_int]
+        f.restype = ctypes.c_int
+        self._bwd = f
 
     # ------------------------------------------------------------------ core
     def rows(self, q, rho, k, v, row_stream, row_nkeys, scale: float,
@@ -168,6 +184,46 @@ class Oracle:
         return out, lse
 
 
+def _probe(self, x, w):
+    """rho = x W_R^T: x [..., K], w [N, K] -> [..., N] (fp64)."""
+    x = _f64(x)
+    w = _f64(w)
+    lead, K = x.shape[:-1], x.shape[-1]
+    N = w.shape[0]
+    assert w.shape == (N, K), "W_R must be [N, K] with K the width of x"
+    xm = np.ascontiguousarray(x.reshape(-1, K))
+    out = np.zeros((xm.shape[0], N), dtype=np.float64)
+    if self._probe(_p(xm), _p(w), _p(out), xm.shape[0], N, K) != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out.reshape(*lead, N)
+
+
+def _prefill_bwd(self, q, rho, k, v, dout, causal: bool, scale: float,
+                 threads: Optional[int] = None):
+    """Gradients of sum(dout * out) for the prefill operator.
+
+    q, rho, dout [B, L, Hq, d]; k, v [B, L, Hkv, d].  Returns (dq, drho, dk,
+    dv) in float64, shaped like q, rho, k, v.
+    """
+    q, rho, k, v, g = (_f64(t) for t in (q, rho, k, v, dout))
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    assert rho.shape == q.shape and g.shape == q.shape and k.shape == (B, L, Hkv, d)
+    assert v.shape == k.shape and Hq % Hkv == 0
+    dq, dr = np.zeros_like(q), np.zeros_like(q)
+    dk, dv = np.zeros_like(k), np.zeros_like(k)
+    rc = self._bwd(_p(q), _p(rho), _p(k), _p(v), _p(g), B, L, Hq, Hkv, d, int(bool(causal)),
+                   float(scale), _p(dq), _p(dr), _p(dk), _p(dv),
+                   int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return dq, dr, dk, dv
+
+
+Oracle.probe = _probe
+Oracle.prefill_bwd = _prefill_bwd
+
+
 def _np(x):
     """numpy view of a numpy array or a (CPU or device) torch tensor, exact values."""
     if isinstance(x, np.ndarray):
@@ -238,3 +294,11 @@ def decode(*args, **kw):
 
 def rows(*args, **kw):
     return get().rows(*args, **kw)
+
+
+def probe(*args, **kw):
+    return get().probe(*args, **kw)
+
+
+def prefill_bwd(*args, **kw):
+    return get().prefill_bwd(*args, **kw)

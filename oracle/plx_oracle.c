@@ -41,6 +41,12 @@
  *
  * Also returned per row: lse = log(sum_j exp(scale * q . k_j)) (natural log).
  * An empty key set gives out = 0 and lse = -inf.
+ *
+ * Two more routines at the end of the file: plxo_probe, the probe projection
+ * rho = W_R x (page 1 section 1.3, page 3), and plxo_prefill_bwd, the
+ * gradients of the prefill operator (derived there; the pages print none),
+ * pinned by finite differences of the forward and by fp64 autograd of the
+ * explicit-covariance definition.
  */
 #include <math.h>
 #include <pthread.h>
@@ -217,5 +223,175 @@ int plxo_rows(const double *q, const double *rho, const double *k,
     for (int t = started + 1; t < nthreads; ++t) plxo_worker(&jobs[t]);
     for (int t = 0; t < nthreads; ++t)
         if (jobs[t].status != 0) return -1;
+    return 0;
+}
+
+/*
+ * plxo_probe: the probe projection rho = W_R x of page 1 section 1.3 ("one
+ * extra projection matrix"; page 3: "rho_i = W_R x_i"), written out.
+ *   x   [M, K]   layer inputs, one row per token
+ *   w   [N, K]   W_R (N = H_q * d output features)
+ *   rho [M, N]   rho[m][n] = sum_k w[n][k] x[m][k]
+ * Returns 0, or -1 on a bad size.
+ */
+int plxo_probe(const double *x, const double *w, double *rho, int64_t M, int64_t N,
+               int64_t K)
+{
+    if (M < 0 || N < 0 || K < 0) return -1;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t kk = 0; kk < K; ++kk) acc += w[n * K + kk] * x[m * K + kk];
+            rho[m * N + n] = acc;
+        }
+    return 0;
+}
+
+/*
+ * Backward of the prefill operator (the pages print no gradient; this is the
+ * derivation, applied to the loss Lo = sum_i g_i . out_i with g = dLo/dout):
+ *
+ *   forward, row i, keys j in J_i:  s_j = scale q.k_j,  a = softmax(s),
+ *     t_j = rho.k_j,  tbar = sum_j a_j t_j,  o = sum_j a_j v_j,
+ *     out = sum_j a_j c_j v_j  with  c_j = 1 + tbar - t_j
+ *     (= o_SA - Sigma_KV^T rho, the explicit form expanded)
+ *   dLo/dv_j   += a_j c_j g
+ *   dLo/dt_j    = a_j (g.o - g.v_j)          (t_j enters c_j and tbar)
+ *   dLo/da_j    = c_j (g.v_j) + t_j (g.o)    (a_j enters out and tbar)
+ *   dLo/ds_j    = a_j (dLo/da_j - sum_m a_m dLo/da_m),
+ *                 sum_m a_m dLo/da_m = g.out + tbar (g.o)
+ *   dLo/dq     += scale sum_j dLo/ds_j k_j
+ *   dLo/drho   += sum_j dLo/dt_j k_j
+ *   dLo/dk_j   += scale dLo/ds_j q + dLo/dt_j rho
+ *
+ * Layouts as the prefill: q, rho, g, dq, drho [B, L, Hq, d]; k, v, dk, dv
+ * [B, L, Hkv, d] (d_k = d_v = d); query head h reads KV head h / (Hq / Hkv);
+ * causal row i sees keys 0..i, otherwise all L.  dk and dv are accumulated
+ * over the rows of all query heads of a KV head, so work is split over
+ * (batch, KV head) pairs.  Returns 0, or -1 on a bad argument.
+ */
+typedef struct {
+    const double *q, *rho, *k, *v, *g;
+    int64_t B, L, Hq, Hkv, d;
+    int causal;
+    double scale;
+    double *dq, *drho, *dk, *dv;
+    int tid, nthreads, status;
+} plxo_bwd_job;
+
+static void *plxo_bwd_worker(void *arg)
+{
+    plxo_bwd_job *jb = (plxo_bwd_job *)arg;
+    const int64_t L = jb->L, Hq = jb->Hq, Hkv = jb->Hkv, d = jb->d, G = Hq / Hkv;
+    double *a = (double *)malloc((size_t)(2 * L + 2 * d + 2) * sizeof(double));
+    if (!a) {
+        jb->status = -1;
+        return NULL;
+    }
+    double *t = a + L, *o = t + L, *outv = o + d;
+    for (int64_t pair = jb->tid; pair < jb->B * Hkv; pair += jb->nthreads) {
+        const int64_t b = pair / Hkv, hk = pair % Hkv;
+#define KROW(j) (jb->k + ((b * L + (j)) * Hkv + hk) * d)
+#define VROW(j) (jb->v + ((b * L + (j)) * Hkv + hk) * d)
+#define DKROW(j) (jb->dk + ((b * L + (j)) * Hkv + hk) * d)
+#define DVROW(j) (jb->dv + ((b * L + (j)) * Hkv + hk) * d)
+        for (int64_t h = hk * G; h < (hk + 1) * G; ++h) {
+            for (int64_t i = 0; i < L; ++i) {
+                const int64_t n = jb->causal ? i + 1 : L;
+                const int64_t ro = ((b * L + i) * Hq + h) * d;
+                const double *qi = jb->q + ro, *ri = jb->rho + ro, *gi = jb->g + ro;
+                /* recompute the forward row */
+                double m = -INFINITY;
+                for (int64_t j = 0; j < n; ++j) {
+                    double s = 0.0, tt = 0.0;
+                    for (int64_t c = 0; c < d; ++c) {
+                        s += qi[c] * KROW(j)[c];
+                        tt += ri[c] * KROW(j)[c];
+                    }
+                    a[j] = jb->scale * s;
+                    t[j] = tt;
+                    if (a[j] > m) m = a[j];
+                }
+                double l = 0.0;
+                for (int64_t j = 0; j < n; ++j) {
+                    a[j] = exp(a[j] - m);
+                    l += a[j];
+                }
+                double tbar = 0.0;
+                for (int64_t j = 0; j < n; ++j) {
+                    a[j] /= l;
+                    tbar += a[j] * t[j];
+                }
+                for (int64_t c = 0; c < d; ++c) o[c] = outv[c] = 0.0;
+                for (int64_t j = 0; j < n; ++j) {
+                    const double cj = 1.0 + tbar - t[j];
+                    for (int64_t c = 0; c < d; ++c) {
+                        o[c] += a[j] * VROW(j)[c];
+                        outv[c] += a[j] * cj * VROW(j)[c];
+                    }
+                }
+                double go = 0.0, gout = 0.0;
+                for (int64_t c = 0; c < d; ++c) {
+                    go += gi[c] * o[c];
+                    gout += gi[c] * outv[c];
+                }
+                const double dsum = gout + tbar * go;  /* sum_m a_m dLo/da_m */
+                double *dqi = jb->dq + ro, *dri = jb->drho + ro;
+                for (int64_t j = 0; j < n; ++j) {
+                    double gv = 0.0;
+                    for (int64_t c = 0; c < d; ++c) gv += gi[c] * VROW(j)[c];
+                    const double cj = 1.0 + tbar - t[j];
+                    const double dt = a[j] * (go - gv);
+                    const double da = cj * gv + t[j] * go;
+                    const double ds = a[j] * (da - dsum);
+                    for (int64_t c = 0; c < d; ++c) {
+                        dqi[c] += jb->scale * ds * KROW(j)[c];
+                        dri[c] += dt * KROW(j)[c];
+                        DKROW(j)[c] += jb->scale * ds * qi[c] + dt * ri[c];
+                        DVROW(j)[c] += a[j] * cj * gi[c];
+                    }
+                }
+            }
+        }
+#undef KROW
+#undef VROW
+#undef DKROW
+#undef DVROW
+    }
+    free(a);
+    jb->status = 0;
+    return NULL;
+}
+
+int plxo_prefill_bwd(const double *q, const double *rho, const double *k, const double *v,
+                     const double *g, int64_t B, int64_t L, int64_t Hq, int64_t Hkv,
+                     int64_t d, int causal, double scale, double *dq, double *drho,
+                     double *dk, double *dv, int nthreads)
+{
+    if (B < 0 || L < 0 || Hq < 1 || Hkv < 1 || d < 1 || Hq % Hkv != 0) return -1;
+    memset(dq, 0, (size_t)(B * L * Hq * d) * sizeof(double));
+    memset(drho, 0, (size_t)(B * L * Hq * d) * sizeof(double));
+    memset(dk, 0, (size_t)(B * L * Hkv * d) * sizeof(double));
+    memset(dv, 0, (size_t)(B * L * Hkv * d) * sizeof(double));
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (B * Hkv < nthreads) nthreads = B * Hkv > 0 ? (int)(B * Hkv) : 1;
+    plxo_bwd_job jobs[256];
+    pthread_t th[256];
+    for (int tt = 0; tt < nthreads; ++tt) {
+        plxo_bwd_job jb = {q, rho, k, v, g, B, L, Hq, Hkv, d, causal, scale,
+                           dq, drho, dk, dv, tt, nthreads, -1};
+        jobs[tt] = jb;
+    }
+    int started = 0;
+    for (int tt = 1; tt < nthreads; ++tt) {
+        if (pthread_create(&th[tt], NULL, plxo_bwd_worker, &jobs[tt]) != 0) break;
+        started = tt;
+    }
+    plxo_bwd_worker(&jobs[0]);
+    for (int tt = 1; tt <= started; ++tt) pthread_join(th[tt], NULL);
+    for (int tt = started + 1; tt < nthreads; ++tt) plxo_bwd_worker(&jobs[tt]);
+    for (int tt = 0; tt < nthreads; ++tt)
+        if (jobs[tt].status != 0) return -1;
     return 0;
 }

@@ -37,6 +37,25 @@ MUTANTS = {
 }
 
 
+# Mistakes in the probe projection and the prefill gradients; each must fail
+# at least one pin of oracle_pins_ext.
+EXT_MUTANTS = {
+    "probe_transposed": ("acc += w[n * K + kk] * x[m * K + kk];",
+                         "acc += w[kk * N + n] * x[m * K + kk];"),
+    "bwd_dt_sign": ("const double dt = a[j] * (go - gv);", "const double dt = a[j] * (gv - go);"),
+    "bwd_dsum_tbar_term_dropped": ("const double dsum = gout + tbar * go;",
+                                   "const double dsum = gout;"),
+    "bwd_da_t_term_dropped": ("const double da = cj * gv + t[j] * go;",
+                              "const double da = cj * gv;"),
+    "bwd_dv_coefficient_dropped": ("DVROW(j)[c] += a[j] * cj * gi[c];",
+                                   "DVROW(j)[c] += a[j] * gi[c];"),
+    "bwd_dk_probe_term_dropped": ("DKROW(j)[c] += jb->scale * ds * qi[c] + dt * ri[c];",
+                                  "DKROW(j)[c] += jb->scale * ds * qi[c];"),
+    "bwd_dq_scale_dropped": ("dqi[c] += jb->scale * ds * KROW(j)[c];",
+                             "dqi[c] += ds * KROW(j)[c];"),
+}
+
+
 @pytest.fixture(scope="module")
 def source():
     with open(SRC) as f:
@@ -70,4 +89,23 @@ def test_mutant_is_caught(source, name):
         O = oracle.Oracle(lib)
         form = "expanded" if name.startswith("expanded") else "explicit"
         caught = _catches(O, form)
+        assert caught, f"mutant {name} passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(EXT_MUTANTS))
+def test_ext_mutant_is_caught(source, name):
+    import oracle_pins_ext
+    old, new = EXT_MUTANTS[name]
+    assert source.count(old) == 1, f"mutant anchor for {name} not unique in oracle source"
+    with tempfile.TemporaryDirectory() as td:
+        src = os.path.join(td, "mutant.c")
+        with open(src, "w") as f:
+            f.write(source.replace(old, new))
+        O = oracle.Oracle(oracle.build(src=src, out=os.path.join(td, "libmutant.so")))
+        caught = []
+        for pin in oracle_pins_ext.ALL_EXT_PINS:
+            try:
+                pin(O)
+            except (AssertionError, ValueError, FloatingPointError) as e:
+                caught.append(f"{pin.__name__}: {str(e)[:80]}")
         assert caught, f"mutant {name} passed every pin"
