@@ -226,7 +226,12 @@ def bench_decode_e2e(plx, W, shape, steps, warmup, world, device, rank):
     """Same metric through the public serving call with host I/O every step: the
     new token's q, rho, k, v and the lengths (which count the new token) are
     packed in one pinned host buffer and copied host -> device in one copy;
-    plx_decode_append writes k, v into the cache and decodes; out comes back."""
+    plx_decode_append writes k, v into the cache and decodes; out comes back to
+    pinned host memory.  As a serving loop would, the copies run on their own
+    stream, double-buffered: step i+1's inputs go up while step i decodes, and
+    step i's output comes down while step i+1 decodes (every step still moves
+    its own inputs and output).  The time runs from the first copy to the last
+    output landing in host memory."""
     import torch
     inp = W.make_decode(shape, seed=100 + rank, device=device, copies=3)
     B, Hq, Hkv, d = shape.B, shape.Hq, shape.Hkv, shape.d
@@ -239,42 +244,60 @@ def bench_decode_e2e(plx, W, shape, steps, warmup, world, device, rank):
         nbytes = t.numel() * t.element_size()
         offs[name] = (off, nbytes, t.dtype, tuple(t.shape))
         off += (nbytes + 255) // 256 * 256
-    hbuf = torch.empty(off, dtype=torch.uint8).pin_memory()
-    for name, t in parts:
-        o, n, _, _ = offs[name]
-        hbuf[o:o + n].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
-    dbuf = torch.empty(off, dtype=torch.uint8, device=device)
-
-    def view(name):
-        o, n, dt, shp = offs[name]
-        return dbuf[o:o + n].view(dt).view(shp)
-
-    q_d, rho_d, kn_d, vn_d, sl_d = (view(n) for n in ("q", "rho", "k", "v", "sl"))
-    out_h = torch.empty((B, Hq, d), dtype=inp["q"].dtype).pin_memory()
-    out_d = torch.empty_like(inp["q"])
+    hbufs, dbufs, outs_h, outs_d, views = [], [], [], [], []
+    for _ in range(2):
+        hbuf = torch.empty(off, dtype=torch.uint8).pin_memory()
+        for name, t in parts:
+            o, n, _, _ = offs[name]
+            hbuf[o:o + n].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
+        dbuf = torch.empty(off, dtype=torch.uint8, device=device)
+        hbufs.append(hbuf)
+        dbufs.append(dbuf)
+        views.append({n_: dbuf[o:o + n].view(dt).view(shp)
+                      for n_, (o, n, dt, shp) in offs.items()})
+        outs_h.append(torch.empty((B, Hq, d), dtype=inp["q"].dtype).pin_memory())
+        outs_d.append(torch.empty_like(inp["q"]))
     ws = plx.decode_workspace(B, Hq, Hkv, d, shape.S_max, device=device)
-    stream = torch.cuda.current_stream()
+    comp = torch.cuda.current_stream()
+    copy = torch.cuda.Stream(device=device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
     def step(i):
-        dbuf.copy_(hbuf, non_blocking=True)
-        plx.decode_append(q_d, rho_d, kn_d, vn_d, inp["k_caches"][i % 3], inp["v_caches"][i % 3],
-                          sl_d, softmax_scale=1.0, out=out_d, workspace=ws, stream=stream)
-        out_h.copy_(out_d, non_blocking=True)
+        b = i % 2
+        v = views[b]
+        with torch.cuda.stream(copy):
+            if i >= 2:
+                copy.wait_event(ev_done[b])  # step i-2 has finished reading this buffer
+            dbufs[b].copy_(hbufs[b], non_blocking=True)
+            ev_in[b].record(copy)
+        comp.wait_event(ev_in[b])
+        if i >= 2:
+            comp.wait_event(ev_out[b])  # step i-2's output has left this buffer
+        plx.decode_append(v["q"], v["rho"], v["k"], v["v"], inp["k_caches"][i % 3],
+                          inp["v_caches"][i % 3], v["sl"], softmax_scale=1.0, out=outs_d[b],
+                          workspace=ws, stream=comp)
+        ev_done[b].record(comp)
+        with torch.cuda.stream(copy):
+            copy.wait_event(ev_done[b])
+            outs_h[b].copy_(outs_d[b], non_blocking=True)
+            ev_out[b].record(copy)
 
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
     barrier(world)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
+    s.record(copy)
     for i in range(steps):
         step(warmup + i)
-    e.record(stream)
+    e.record(copy)  # after the last output's copy to the host
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world, device)
-    h2d = hbuf.numel()
-    d2h = out_h.numel() * out_h.element_size()
+    h2d = hbufs[0].numel()
+    d2h = outs_h[0].numel() * outs_h[0].element_size()
     return {"ms": ms, "h2d": h2d, "d2h": d2h}
 
 

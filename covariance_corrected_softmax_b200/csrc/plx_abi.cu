@@ -67,7 +67,9 @@ cudaError_t get_encoder() {
   return g_encode ? cudaSuccess : cudaErrorNotSupported;
 }
 
-// 4-D map over a [B, S, H, D] tensor, box (D, 1, box_rows, 1), no swizzle.
+// 4-D map over a [B, S, H, D] tensor, box (box_cols, 1, box_rows, 1): bf16
+// boxes of 64 columns with the 128-byte swizzle, fp32 boxes of full rows with
+// none (plx::decode_box_cols).
 cudaError_t encode_rows_map(CUtensorMap* map, const void* base, bool bf16, int B, int S, int H,
                             int D, int box_rows) {
   cudaError_t e = get_encoder();
@@ -75,11 +77,12 @@ cudaError_t encode_rows_map(CUtensorMap* map, const void* base, bool bf16, int B
   const cuuint64_t esz = bf16 ? 2 : 4;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
   cuuint64_t strides[3] = {D * esz, (cuuint64_t)H * D * esz, (cuuint64_t)S * H * D * esz};
-  cuuint32_t box[4] = {(cuuint32_t)D, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t box[4] = {(cuuint32_t)plx::decode_box_cols(bf16, D), 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                         4, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -170,6 +173,32 @@ size_t plx_decode_workspace_bytes(int B, int H_q, int H_kv, int d, int S_max) {
 
 namespace {
 
+plx_status prefill_impl(const void* q, const void* rho, const void* k, const void* v, void* out,
+                        float* lse, int causal, int B, int L, int H_q, int H_kv, int d,
+                        plx_dtype dtype, plx_dtype out_dtype, float softmax_scale, void* stream,
+                        bool check_only);
+
+// rho[M, N] = x[M, K] w_r[N, K]^T (all checks first; check_only stops there).
+plx_status projection_impl(const void* x, const void* w_r, void* rho, int M, int N, int K,
+                           plx_dtype dtype, void* stream, bool check_only) {
+  t_last_cuda_error = 0;
+  if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
+  if (M < 0 || N < 0 || K < 1) return PLX_ERR_INVALID_ARGUMENT;
+  if (M == 0 || N == 0) return PLX_OK;
+  if (!x || !w_r || !rho || !aligned16(x) || !aligned16(w_r) || !aligned16(rho))
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (dtype == PLX_BF16 && (K % 8 != 0 || N % 8 != 0)) return PLX_ERR_UNSUPPORTED;
+  if (check_only) return PLX_OK;
+  int sms = 0;
+  unsigned* err = nullptr;
+  cudaError_t e = device_info(&sms, &err);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = plx::launch_probe_projection(x, w_r, rho, M, N, K, dtype == PLX_BF16, sms, err,
+                                   static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return PLX_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? PLX_OK : cuda_fail(e);
+}
+
 // plx_decode, preceded (when k_new is given) by the KV-cache append of
 // plx_decode_append.  Every check runs before the first launch.
 // Paged caches (block_table != nullptr): k_cache, v_cache are the page pools
@@ -183,7 +212,8 @@ plx_status decode_impl(const void* q, const void* rho, const void* k_new, const 
                        const void* k_cache, const void* v_cache, const int32_t* seqlens,
                        void* out, int B, int H_q, int H_kv, int d, int S_max, plx_dtype dtype,
                        float softmax_scale, void* workspace, size_t workspace_bytes,
-                       void* stream, const Paging& pg = Paging(), float* state = nullptr) {
+                       void* stream, const Paging& pg = Paging(), float* state = nullptr,
+                       bool check_only = false) {
   t_last_cuda_error = 0;
   if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
   if (B < 0 || S_max < 1 || !shape_ok(H_q, H_kv, d)) return PLX_ERR_INVALID_ARGUMENT;
@@ -213,16 +243,21 @@ plx_status decode_impl(const void* q, const void* rho, const void* k_new, const 
   const long long max_tiles = (long long)B * H_kv * (G / hpw) * ((S_max + tk - 1) / tk);
   const int grid = (int)(max_tiles < sms ? max_tiles : sms);
   if (workspace_bytes < decode_ws_bytes_for(d, hpw, sms)) return PLX_ERR_WORKSPACE_TOO_SMALL;
+  if (check_only) return PLX_OK;
 
-  CUtensorMap kmap, vmap;
+  plx::DecodeMaps maps;
   if (pg.block_table) {
     // one [num_pages * page_size, H_kv, d] pool, 16-row boxes
     const int rows = pg.num_pages * pg.page_size;
-    e = encode_rows_map(&kmap, k_cache, bf16, 1, rows, H_kv, d, 16);
-    if (e == cudaSuccess) e = encode_rows_map(&vmap, v_cache, bf16, 1, rows, H_kv, d, 16);
+    e = encode_rows_map(&maps.k_chunk, k_cache, bf16, 1, rows, H_kv, d, 16);
+    if (e == cudaSuccess) e = encode_rows_map(&maps.v_chunk, v_cache, bf16, 1, rows, H_kv, d, 16);
+    maps.k = maps.k_chunk;  // unused by the paged kernel
+    maps.v = maps.v_chunk;
   } else {
-    e = encode_rows_map(&kmap, k_cache, bf16, B, S_max, H_kv, d, tk);
-    if (e == cudaSuccess) e = encode_rows_map(&vmap, v_cache, bf16, B, S_max, H_kv, d, tk);
+    e = encode_rows_map(&maps.k, k_cache, bf16, B, S_max, H_kv, d, tk);
+    if (e == cudaSuccess) e = encode_rows_map(&maps.v, v_cache, bf16, B, S_max, H_kv, d, tk);
+    if (e == cudaSuccess) e = encode_rows_map(&maps.k_chunk, k_cache, bf16, B, S_max, H_kv, d, 16);
+    if (e == cudaSuccess) e = encode_rows_map(&maps.v_chunk, v_cache, bf16, B, S_max, H_kv, d, 16);
   }
   if (e != cudaSuccess) return cuda_fail(e);
 
@@ -253,7 +288,7 @@ plx_status decode_impl(const void* q, const void* rho, const void* k_new, const 
   p.page_size = pg.page_size;
   p.max_pages = pg.max_pages;
   p.state = state;
-  e = plx::launch_decode(bf16, d, kmap, vmap, p, hpw, st);
+  e = plx::launch_decode(bf16, d, maps, p, hpw, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return PLX_OK;
 }
@@ -397,6 +432,18 @@ plx_status plx_prefill_fwd_ex(const void* q, const void* rho, const void* k, con
                               void* out, float* lse, int causal, int B, int L, int H_q, int H_kv,
                               int d, plx_dtype dtype, plx_dtype out_dtype, float softmax_scale,
                               void* stream) {
+  return prefill_impl(q, rho, k, v, out, lse, causal, B, L, H_q, H_kv, d, dtype, out_dtype,
+                      softmax_scale, stream, false);
+}
+
+}  // extern "C"
+
+namespace {
+
+plx_status prefill_impl(const void* q, const void* rho, const void* k, const void* v, void* out,
+                        float* lse, int causal, int B, int L, int H_q, int H_kv, int d,
+                        plx_dtype dtype, plx_dtype out_dtype, float softmax_scale, void* stream,
+                        bool check_only) {
   t_last_cuda_error = 0;
   if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
   if (out_dtype != dtype && !(dtype == PLX_BF16 && out_dtype == PLX_F32))
@@ -411,6 +458,7 @@ plx_status plx_prefill_fwd_ex(const void* q, const void* rho, const void* k, con
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return PLX_ERR_INVALID_ARGUMENT;
   if ((long long)B * L > (1ll << 31) || B > 65535 || H_q > 65535) return PLX_ERR_UNSUPPORTED;
+  if (check_only) return PLX_OK;
 
   int sms = 0;
   unsigned* err = nullptr;
@@ -457,4 +505,93 @@ plx_status plx_prefill_fwd_ex(const void* q, const void* rho, const void* k, con
   return e == cudaSuccess ? PLX_OK : cuda_fail(e);
 }
 
+}  // namespace
+
+extern "C" {
+
+plx_status plx_probe_projection(const void* x, const void* w_r, void* rho, int M, int N, int K,
+                                plx_dtype dtype, void* stream) {
+  return projection_impl(x, w_r, rho, M, N, K, dtype, stream, false);
+}
+
+plx_status plx_prefill_fwd_x(const void* q, const void* x, const void* w_r, const void* k,
+                             const void* v, void* rho, void* out, float* lse, int causal, int B,
+                             int L, int H_q, int H_kv, int d, int d_model, plx_dtype dtype,
+                             float softmax_scale, void* stream) {
+  // every argument of both steps is checked before the first launch
+  if (B < 0 || L < 0 || !shape_ok(H_q, H_kv, d) || d_model < 1) {
+    t_last_cuda_error = 0;
+    return PLX_ERR_INVALID_ARGUMENT;
+  }
+  const long long M = (long long)B * L;
+  if (M > 0x7fffffffll || (long long)H_q * d > 0x7fffffffll) {
+    t_last_cuda_error = 0;
+    return PLX_ERR_UNSUPPORTED;
+  }
+  plx_status s = projection_impl(x, w_r, rho, (int)M, H_q * d, d_model, dtype, stream, true);
+  if (s == PLX_OK)
+    s = prefill_impl(q, rho, k, v, out, lse, causal, B, L, H_q, H_kv, d, dtype, dtype,
+                     softmax_scale, stream, true);
+  if (s != PLX_OK || M == 0) return s;
+  s = projection_impl(x, w_r, rho, (int)M, H_q * d, d_model, dtype, stream, false);
+  if (s != PLX_OK) return s;
+  return prefill_impl(q, rho, k, v, out, lse, causal, B, L, H_q, H_kv, d, dtype, dtype,
+                      softmax_scale, stream, false);
+}
+
+plx_status plx_decode_x(const void* q, const void* x, const void* w_r, const void* k_cache,
+                        const void* v_cache, const int32_t* seqlens, void* rho, void* out, int B,
+                        int H_q, int H_kv, int d, int S_max, int d_model, plx_dtype dtype,
+                        float softmax_scale, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  if (B < 0 || !shape_ok(H_q, H_kv, d) || d_model < 1) {
+    t_last_cuda_error = 0;
+    return PLX_ERR_INVALID_ARGUMENT;
+  }
+  plx_status s = projection_impl(x, w_r, rho, B, H_q * d, d_model, dtype, stream, true);
+  if (s == PLX_OK)
+    s = decode_impl(q, rho, nullptr, nullptr, k_cache, v_cache, seqlens, out, B, H_q, H_kv, d,
+                    S_max, dtype, softmax_scale, workspace, workspace_bytes, stream, Paging(),
+                    nullptr, true);
+  if (s != PLX_OK || B == 0) return s;
+  s = projection_impl(x, w_r, rho, B, H_q * d, d_model, dtype, stream, false);
+  if (s != PLX_OK) return s;
+  return decode_impl(q, rho, nullptr, nullptr, k_cache, v_cache, seqlens, out, B, H_q, H_kv, d,
+                     S_max, dtype, softmax_scale, workspace, workspace_bytes, stream);
+}
+
+size_t plx_prefill_bwd_workspace_bytes(int B, int L, int H_q) {
+  if (B < 0 || L < 0 || H_q < 1) return 0;
+  return plx::prefill_bwd_workspace_bytes(B, L, H_q);
+}
+
+plx_status plx_prefill_bwd(const void* q, const void* rho, const void* k, const void* v,
+                           const void* dout, float* dq, float* drho, float* dk, float* dv,
+                           int causal, int B, int L, int H_q, int H_kv, int d, plx_dtype dtype,
+                           float softmax_scale, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  t_last_cuda_error = 0;
+  if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARGUMENT;
+  if (B < 0 || L < 0 || !shape_ok(H_q, H_kv, d) || (causal != 0 && causal != 1))
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (B == 0 || L == 0) return PLX_OK;
+  if (!q || !rho || !k || !v || !dout || !dq || !drho || !dk || !dv || !workspace)
+    return PLX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(rho) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(drho) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(workspace))
+    return PLX_ERR_INVALID_ARGUMENT;
+  if ((long long)B * L * H_q > 0x7fffffffll * 8) return PLX_ERR_UNSUPPORTED;
+  if (workspace_bytes < plx::prefill_bwd_workspace_bytes(B, L, H_q))
+    return PLX_ERR_WORKSPACE_TOO_SMALL;
+  const cudaError_t e = plx::launch_prefill_bwd(q, rho, k, v, dout, dq, drho, dk, dv, workspace,
+                                                causal, B, L, H_q, H_kv, d, dtype == PLX_BF16,
+                                                softmax_scale, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PLX_OK : cuda_fail(e);
+}
+
 }  // extern "C"
+
+

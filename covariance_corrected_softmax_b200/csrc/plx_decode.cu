@@ -137,22 +137,130 @@ __device__ void locate_range(const DecodeParams& p, int TK, RangeInfo* info, lon
 }
 
 // ---------------------------------------------------------------------------
+// Warp-level tensor-core helpers (bf16 consumers).
+// ---------------------------------------------------------------------------
+// Four 8x8 b16 matrices from shared memory; lanes 8j..8j+7 give the row
+// addresses of matrix j; register j of lane L holds row L/4, elements
+// 2(L%4), 2(L%4)+1 of matrix j (the .trans form: the transposed matrix).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+// c (16x8 fp32) += a (16x16 bf16, row-major) * b (16x8 bf16, column-major).
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk c (8 bf16 elements) of row `row` in a tile of
+// 64-column boxes with the 128-byte swizzle (chunk index XOR row mod 8).
+template <int BOX_BYTES>
+__device__ __forceinline__ uint32_t swz_off(int row, int c) {
+  return (uint32_t)((c >> 3) * BOX_BYTES + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+}
+
+// Kernel instances (see the main kernel).
+constexpr int kDecContiguous = 0, kDecPaged = 1, kDecState = 2;
+constexpr int kDecStateMode = kDecState;
+
+// ---------------------------------------------------------------------------
+// Segment finalisation: merge the NW consumer warps' states of a head group
+// (in shared memory: [warp][head] m, l, z, pad, o[D], u[D]) with the
+// log-sum-exp rule, then write the output (a segment complete in this CTA),
+// the row's softmax state (state mode), or this CTA's partial slot with its
+// header (a segment split across CTAs; the combine kernel merges the pieces).
+// Called by all consumer threads between two consumer-wide barriers.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int HPW, int MODE, int NW>
+__device__ __forceinline__ void finalize_segment(const DecodeParams& p, const TileMeta& mt, int h0,
+                                                 bool complete, float* part,
+                                                 const float* merge, int tid) {
+  constexpr int PHF = part_head_floats<D>();
+  for (int pr = tid; pr < HPW * D; pr += NW * 32) {
+    const int g = pr / D, c = pr % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, merge[(w * HPW + g) * PHF]);
+    float L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float* src = merge + (w * HPW + g) * PHF;
+      const float wt = merge_weight(src[0], M);
+      L += wt * src[1];
+      Z += wt * src[2];
+      O += wt * src[4 + c];
+      U += wt * src[4 + D + c];
+    }
+    if (MODE == kDecStateMode && complete) {
+      float* sr = p.state + ((size_t)mt.b * p.Hq + h0 + g) * PHF;
+      if (c == 0) {
+        sr[0] = M;
+        sr[1] = L;
+        sr[2] = Z;
+        sr[3] = 0.f;
+      }
+      sr[4 + c] = O;
+      sr[4 + D + c] = U;
+    } else if (complete) {
+      // out = (1 + tbar) o - u with tbar = Z/L, o = O/L, u = U/L
+      const float inv = 1.f / L;
+      const float val = ((1.f + Z * inv) * O - U) * inv;
+      store_elem<T>(p.out, ((size_t)mt.b * p.Hq + h0 + g) * D + c, val);
+    } else {
+      float* ph = part + kPartHeader + g * PHF;
+      if (c == 0) {
+        ph[0] = M;
+        ph[1] = L;
+        ph[2] = Z;
+      }
+      ph[4 + c] = O;
+      ph[4 + D + c] = U;
+    }
+  }
+  if (!complete && tid == 0) {
+    int* hdr = reinterpret_cast<int*>(part);
+    hdr[1] = (mt.flags & 4) ? 1 : 0;
+    hdr[2] = (mt.flags & 8) ? 1 : 0;
+    hdr[3] = 0;
+    hdr[0] = mt.seg;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Main decode kernel.
 // ---------------------------------------------------------------------------
 // MODE: kDecContiguous, kDecPaged (block-table loads), kDecState (contiguous
 // loads, softmax states written instead of the output).  Each is a separate
 // instance, so the common one carries no code of the others.
-constexpr int kDecContiguous = 0, kDecPaged = 1, kDecState = 2;
 
+// kmap, vmap: TK-row boxes over the contiguous cache (unused when paged).
+// kmap_c, vmap_c: 16-row boxes over the contiguous cache (a segment's last,
+// partial tile) or over the page pools (paged).
 template <typename T, int D, int HPW, int MODE>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     plx_decode_splitk_kernel(const __grid_constant__ CUtensorMap kmap,
-                             const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+                             const __grid_constant__ CUtensorMap vmap,
+                             const __grid_constant__ CUtensorMap kmap_c,
+                             const __grid_constant__ CUtensorMap vmap_c, const DecodeParams p) {
   using Cfg = DecodeTile<T, D>;
-  constexpr int TK = Cfg::TK, KPH = Cfg::KPH, EPL = Cfg::EPL, STAGES = Cfg::STAGES;
+  constexpr int NW = Cfg::NW, TK = Cfg::TK, KPH = Cfg::KPH, EPL = Cfg::EPL,
+                STAGES = Cfg::STAGES, CB = Cfg::CB;
   constexpr int H2 = EPL / 2;
   constexpr int PF = part_floats<D>(HPW);
   constexpr int PHF = part_head_floats<D>();
+  constexpr int CH = kDecChunkRows;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -166,8 +274,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(scan_ws + 16);
   float* merge = reinterpret_cast<float*>(scan_ws + 20);
   float* red_smem = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(merge + kDecConsumerWarps * HPW * PHF) + 15) & ~uintptr_t(15));
-  float* bc_smem = red_smem + 2 * kDecConsumerWarps * kDecRedRegion;
+      (reinterpret_cast<uintptr_t>(merge + NW * HPW * PHF) + 15) & ~uintptr_t(15));
+  float* bc_smem = red_smem + 2 * NW * kDecRedRegion;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -180,7 +288,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     s1[0] = -1;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kDecConsumerWarps);
+      mbar_init(&empty[s], NW);
     }
     fence_mbarrier_init();
   }
@@ -206,71 +314,33 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const long long t0 = info->t0, t1 = info->t1;
   const int segs_per_b = p.Hkv * p.nhg;
 
-  if (warp == kDecConsumerWarps) {
+  if (warp == NW) {
     // ------------------------------------------------------------ producer
-    if constexpr (MODE != kDecPaged) {
-      // contiguous cache: one lane issues one K and one V load per tile
-      if (lane == 0 && t0 < t1) {
-        tma_prefetch_desc(&kmap);
-        tma_prefetch_desc(&vmap);
-        int b = info->b0;
-        int len = clamp_len(p.seqlens[b], p.S_max);
-        int nt = (len + TK - 1) / TK;
-        int seg_local = (int)(info->off0 / nt);
-        int kt = (int)(info->off0 % nt);
-        bool starts_here = (kt == 0);
-        for (long long t = t0, i = 0; t < t1; ++t, ++i) {
-          const int stage = (int)(i % STAGES);
-          if (i >= STAGES) {
-            if (!mbar_wait(&empty[stage], (uint32_t)(((i / STAGES) - 1) & 1), abort_flag, p.err)) break;
-          }
-          TileMeta m;
-          m.b = b;
-          m.hkv = seg_local / p.nhg;
-          m.hg = seg_local % p.nhg;
-          m.kt = kt;
-          m.nvalid = min(TK, len - kt * TK);
-          m.seg = b * segs_per_b + seg_local;
-          m.flags = ((t == t0 || kt == 0) ? 1 : 0) | ((t == t1 - 1 || kt == nt - 1) ? 2 : 0) |
-                    (starts_here ? 4 : 0) | ((kt == nt - 1) ? 8 : 0);
-          m.pad = 0;
-          metas[stage] = m;
-          mbar_arrive_expect_tx(&full[stage], 2 * Cfg::TILE_BYTES);
-          uint8_t* dst = ring + stage * Cfg::STAGE_BYTES;
-          tma_load_4d(dst, &kmap, &full[stage], 0, m.hkv, kt * TK, b);
-          tma_load_4d(dst + Cfg::TILE_BYTES, &vmap, &full[stage], 0, m.hkv, kt * TK, b);
-          // advance the walk
-          if (++kt == nt) {
-            kt = 0;
-            starts_here = true;
-            if (++seg_local == segs_per_b) {
-              seg_local = 0;
-              do {
-                ++b;
-              } while (b < p.B && clamp_len(p.seqlens[b], p.S_max) == 0);
-              if (b < p.B) {
-                len = clamp_len(p.seqlens[b], p.S_max);
-                nt = (len + TK - 1) / TK;
-              }
-            }
-          }
+    // The tile walk (batch-major over (batch, kv-head, head-group) segments,
+    // tiles of TK keys, from this CTA's first tile t0) runs in every lane.
+    if (t0 < t1) {
+      int b = info->b0;
+      int len = clamp_len(p.seqlens[b], p.S_max);
+      int nt = (len + TK - 1) / TK;
+      int seg_local = (int)(info->off0 / nt);
+      int kt = (int)(info->off0 % nt);
+      bool starts_here = (kt == 0);
+      if (lane == 0) {
+        tma_prefetch_desc(&kmap_c);
+        tma_prefetch_desc(&vmap_c);
+        if constexpr (MODE != kDecPaged) {
+          tma_prefetch_desc(&kmap);
+          tma_prefetch_desc(&vmap);
         }
       }
-    } else if (t0 < t1) {
-      // The same tile walk as above (batch-major over (batch, kv-head,
-      // head-group) segments, tiles of TK keys, from this CTA's first tile t0),
-      // run by every lane of the warp.
-      int b = 0, len = 0, nt = 1, seg_local = 0, kt = 0;
-      bool starts_here = false;
-      auto walk_init = [&]() {
-        b = info->b0;
-        len = clamp_len(p.seqlens[b], p.S_max);
-        nt = (len + TK - 1) / TK;
-        seg_local = (int)(info->off0 / nt);
-        kt = (int)(info->off0 % nt);
-        starts_here = (kt == 0);
-      };
-      auto tile_meta = [&](long long t) {
+      for (long long t = t0, i = 0; t < t1; ++t, ++i) {
+        const int stage = (int)(i % STAGES);
+        if (i >= STAGES) {
+          int okw = 1;
+          if (lane == 0)
+            okw = mbar_wait(&empty[stage], (uint32_t)(((i / STAGES) - 1) & 1), abort_flag, p.err);
+          if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+        }
         TileMeta m;
         m.b = b;
         m.hkv = seg_local / p.nhg;
@@ -281,9 +351,58 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         m.flags = ((t == t0 || kt == 0) ? 1 : 0) | ((t == t1 - 1 || kt == nt - 1) ? 2 : 0) |
                   (starts_here ? 4 : 0) | ((kt == nt - 1) ? 8 : 0);
         m.pad = 0;
-        return m;
-      };
-      auto walk_next = [&]() {
+        uint8_t* dst = ring + stage * Cfg::STAGE_BYTES;
+        // Paged caches always, and (bf16) a partial last tile, come in 16-row
+        // chunks: lane c loads chunk c; chunks past the length are not loaded
+        // (the consumers mask their rows).
+        const bool chunked = MODE == kDecPaged || (Cfg::MMA && m.nvalid < TK);
+        if (!chunked) {
+          if (lane == 0) {
+            metas[stage] = m;
+            mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+#pragma unroll
+            for (int cb = 0; cb < CB; ++cb) {
+              tma_load_4d(dst + cb * Cfg::BOX_BYTES, &kmap, &full[stage], cb * 64, m.hkv,
+                          kt * TK, b);
+              tma_load_4d(dst + Cfg::TILE_BYTES + cb * Cfg::BOX_BYTES, &vmap, &full[stage],
+                          cb * 64, m.hkv, kt * TK, b);
+            }
+          }
+        } else {
+          const int nch = (m.nvalid + CH - 1) / CH;
+          const int c = lane;
+          int row = -CH, bc = b;
+          if (c < nch) {
+            const int pos = kt * TK + CH * c;
+            if constexpr (MODE == kDecPaged) {
+              // a page index outside the pool is reported and read as zeros
+              // (out-of-range TMA rows)
+              const int page = p.block_table[(size_t)b * p.max_pages + pos / p.page_size];
+              bc = 0;
+              if (page >= 0 && page < p.num_pages)
+                row = page * p.page_size + pos % p.page_size;
+              else
+                record_error(p.err, kDevBadArgument);
+            } else {
+              row = pos;
+            }
+          }
+          if (lane == 0) {
+            metas[stage] = m;
+            mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * nch * CH * Cfg::ROW_BYTES));
+          }
+          __syncwarp();
+          if (c < nch) {
+#pragma unroll
+            for (int cb = 0; cb < CB; ++cb) {
+              const int off = cb * Cfg::BOX_BYTES + c * CH * Cfg::BOX_ROW;
+              tma_load_4d(dst + off, &kmap_c, &full[stage], cb * 64, m.hkv, row, bc);
+              tma_load_4d(dst + Cfg::TILE_BYTES + off, &vmap_c, &full[stage], cb * 64, m.hkv,
+                          row, bc);
+            }
+          }
+        }
+        // advance the walk
         if (++kt == nt) {
           kt = 0;
           starts_here = true;
@@ -298,54 +417,204 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
           }
         }
-      };
-      // Paged cache: 16-row chunks, each inside one page (page_size is a
-      // multiple of 16).  The whole warp walks the tiles; lane c looks up and
-      // loads chunk c, so the block-table reads of a tile go out together.
-      // Chunks past the length are not loaded (the consumers mask their rows);
-      // a page index outside the pool is reported and read as zeros
-      // (out-of-range TMA rows).
-      if (lane == 0) {
-        tma_prefetch_desc(&kmap);
-        tma_prefetch_desc(&vmap);
       }
-      walk_init();
-      for (long long t = t0, i = 0; t < t1; ++t, ++i) {
-        const int stage = (int)(i % STAGES);
-        if (i >= STAGES) {
-          int okw = 1;
-          if (lane == 0)
-            okw = mbar_wait(&empty[stage], (uint32_t)(((i / STAGES) - 1) & 1), abort_flag, p.err);
-          if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+    }
+  } else if constexpr (Cfg::MMA) {
+    // ------------------------------------------------------------ consumers (bf16)
+    // Warp w owns keys [16w, 16w + 16) of every tile.  Lane L = 4g + tq:
+    //  score chain: A rows g = q of head hh, g + 8 = rho of head hh; C holds,
+    //    for keys 8nb + 2tq + {0, 1} (nb = 0, 1), q.k in c0, c1 and rho.k in
+    //    c2, c3;
+    //  weights: B row (kind) g of the value product: p (kinds with bit 1
+    //    clear) or p t (bit 1 set) of head hh, its bf16 high part (g < 4) or
+    //    the bf16 rounding of the remainder (g >= 4); for keys 2tq + {0, 1}
+    //    (b0) and 8 + 2tq + {0, 1} (b1): the very keys of the score fragment;
+    //  value accumulators acc[mb]: head dims 16mb + g (c0, c1) and + 8 (c2, c3)
+    //    of kinds 2tq (head 0) and 2tq + 1 (head 1): tq = 0 the high parts of
+    //    o, 1 of u, 2 the low parts of o, 3 of u.
+    constexpr int KS = D / 16;
+    const int g = lane >> 2, tq = lane & 3;
+    const int hh = HPW == 2 ? (g & 1) : 0;
+    const bool w_pt = ((g >> 1) & 1) != 0;
+    const bool w_lo = g >= 4;
+    const bool w_live = HPW == 2 || (g & 1) == 0;  // one head: odd kinds unused
+    const int lj = lane >> 3, lr = lane & 7;       // ldmatrix: matrix, row
+    const int kw0 = warp * 16;                     // this warp's first key of a tile
+    const uint32_t ring_s = smem_u32(ring);
+    uint32_t qa[KS][4];
+    float acc[KS][4];
+    float m_run = -INFINITY, lsum = 0.f, zsum = 0.f;
+    int ordinal = 0;  // segments finalised so far by this CTA
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qa[ks][e] = 0u;
+        acc[ks][e] = 0.f;
+      }
+
+    for (long long t = t0, i = 0; t < t1; ++t, ++i) {
+      const int stage = (int)(i % STAGES);
+      if (!mbar_wait(&full[stage], (uint32_t)((i / STAGES) & 1), abort_flag, p.err)) break;
+      const TileMeta mt = metas[stage];
+      const int h0 = mt.hkv * p.G + mt.hg * HPW;  // first query head of the group
+
+      if (mt.flags & 1) {  // first tile of a segment in this CTA: load q, rho; reset
+        const size_t row = ((size_t)mt.b * p.Hq + h0 + hh) * (D / 2);
+        const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q) + row;
+        const uint32_t* r32 = reinterpret_cast<const uint32_t*>(p.rho) + row;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qa[ks][0] = q32[8 * ks + tq];
+          qa[ks][1] = r32[8 * ks + tq];
+          qa[ks][2] = q32[8 * ks + 4 + tq];
+          qa[ks][3] = r32[8 * ks + 4 + tq];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[ks][e] = 0.f;
         }
-        const TileMeta m = tile_meta(t);
-        uint8_t* dst = ring + stage * Cfg::STAGE_BYTES;
-        const int nch = (m.nvalid + 15) >> 4;
-        const int c = lane;
-        int row = -16;
-        if (c < nch) {
-          const int pos = kt * TK + 16 * c;
-          const int page = p.block_table[(size_t)b * p.max_pages + pos / p.page_size];
-          if (page >= 0 && page < p.num_pages)
-            row = page * p.page_size + pos % p.page_size;
-          else
-            record_error(p.err, kDevBadArgument);
+        m_run = -INFINITY;
+        lsum = zsum = 0.f;
+      }
+
+      const int nv = mt.nvalid - kw0;  // valid keys of this warp in the tile
+      if (nv > 0) {
+        const uint32_t kbase = ring_s + stage * Cfg::STAGE_BYTES;
+        const uint32_t vbase = kbase + Cfg::TILE_BYTES;
+        // scores: cs[nb] = [q; rho] x K^T for keys kw0 + 8nb .. + 7
+        float cs[2][4];
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          cs[nb][0] = cs[nb][1] = cs[nb][2] = cs[nb][3] = 0.f;
+          const int key = kw0 + 8 * nb + lr;
+#pragma unroll
+          for (int kp = 0; kp < KS / 2; ++kp) {
+            uint32_t bk[4];
+            ldsm_x4(kbase + swz_off<Cfg::BOX_BYTES>(key, 4 * kp + lj), bk);
+            mma_bf16_16816(cs[nb], qa[2 * kp], bk[0], bk[1]);
+            mma_bf16_16816(cs[nb], qa[2 * kp + 1], bk[2], bk[3]);
+          }
         }
-        if (lane == 0) {
-          metas[stage] = m;
-          mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * nch * 16 * Cfg::ROW_BYTES));
+        // this lane's keys: 2tq, 2tq + 1, 8 + 2tq, 9 + 2tq (of the warp's 16)
+        float sv[4] = {cs[0][0] * p.qscale, cs[0][1] * p.qscale, cs[1][0] * p.qscale,
+                       cs[1][1] * p.qscale};
+        float tv[4] = {cs[0][2], cs[0][3], cs[1][2], cs[1][3]};
+        const bool tail = nv < 16;
+        if (tail) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            if (8 * (kk >> 1) + 2 * tq + (kk & 1) >= nv) {
+              sv[kk] = -INFINITY;
+              tv[kk] = 0.f;  // rows past the length may hold anything
+            }
         }
-        __syncwarp();
-        if (c < nch) {
-          tma_load_4d(dst + c * 16 * Cfg::ROW_BYTES, &kmap, &full[stage], 0, m.hkv, row, 0);
-          tma_load_4d(dst + Cfg::TILE_BYTES + c * 16 * Cfg::ROW_BYTES, &vmap, &full[stage], 0,
-                      m.hkv, row, 0);
+        float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        // lazy running max of head hh: moves only when the tile's max exceeds
+        // it by more than 2^8, so every weight stays <= 2^8
+        float alpha = 1.f;
+        if (mx > m_run + 8.f) {
+          alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - mx);
+          m_run = mx;
         }
-        walk_next();
+        const float alpha_x = __shfl_xor_sync(0xffffffffu, alpha, 4);  // the other head's
+        const float a0 = (HPW == 1 || hh == 0) ? alpha : alpha_x;
+        const float a1 = (HPW == 2 && hh == 1) ? alpha : alpha_x;
+        if (a0 != 1.f || a1 != 1.f) {
+#pragma unroll
+          for (int mb = 0; mb < KS; ++mb) {
+            acc[mb][0] *= a0;
+            acc[mb][1] *= a1;
+            acc[mb][2] *= a0;
+            acc[mb][3] *= a1;
+          }
+        }
+        lsum *= alpha;
+        zsum *= alpha;
+        float w[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const float pp = fast_exp2(sv[kk] - m_run);  // 0 for a masked key
+          const float pt = pp * tv[kk];
+          lsum += pp;
+          zsum += pt;
+          w[kk] = w_pt ? pt : pp;
+        }
+        uint32_t bw[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t hi = float2_to_bf16x2(w[2 * h], w[2 * h + 1]);
+          if (w_lo) {
+            const float2 hf = bf16x2_to_float2(hi);
+            bw[h] = float2_to_bf16x2(w[2 * h] - hf.x, w[2 * h + 1] - hf.y);
+          } else {
+            bw[h] = hi;
+          }
+          if (!w_live) bw[h] = 0u;
+        }
+        // value products: acc[mb] += V^T[16mb.., keys] x W^T
+        uint32_t mk01 = 0xffffffffu, mk23 = 0xffffffffu;
+        if (tail) {
+          mk01 = (2 * tq < nv ? 0x0000ffffu : 0u) | (2 * tq + 1 < nv ? 0xffff0000u : 0u);
+          mk23 = (2 * tq + 8 < nv ? 0x0000ffffu : 0u) | (2 * tq + 9 < nv ? 0xffff0000u : 0u);
+        }
+        const int vkey = kw0 + 8 * (lj >> 1) + lr;
+#pragma unroll
+        for (int mb = 0; mb < KS; ++mb) {
+          uint32_t av[4];
+          ldsm_x4_trans(vbase + swz_off<Cfg::BOX_BYTES>(vkey, 2 * mb + (lj & 1)), av);
+          av[0] &= mk01;
+          av[1] &= mk01;
+          av[2] &= mk23;
+          av[3] &= mk23;
+          mma_bf16_16816(acc[mb], av, bw[0], bw[1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+
+      if (mt.flags & 2) {
+        // ---- this warp's state of the segment, to shared memory
+        float ls = lsum, zs = zsum;
+        ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+        ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+        zs += __shfl_xor_sync(0xffffffffu, zs, 1);
+        zs += __shfl_xor_sync(0xffffffffu, zs, 2);
+        float* dstw = merge + warp * HPW * PHF;
+#pragma unroll
+        for (int mb = 0; mb < KS; ++mb) {
+          float o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[e] = acc[mb][e] + __shfl_xor_sync(0xffffffffu, acc[mb][e], 2);
+          if (tq < 2) {  // tq 0: o (high + low parts), tq 1: u
+            const int off = 4 + tq * D + 16 * mb + g;
+            dstw[off] = o[0];
+            dstw[off + 8] = o[2];
+            if (HPW == 2) {
+              dstw[PHF + off] = o[1];
+              dstw[PHF + off + 8] = o[3];
+            }
+          }
+        }
+        if (tq == 0 && g < HPW) {
+          dstw[g * PHF + 0] = m_run;
+          dstw[g * PHF + 1] = ls;
+          dstw[g * PHF + 2] = zs;
+        }
+      }
+      if (mt.flags & 2) {
+        named_bar_sync(1, NW * 32);
+        const bool complete = (mt.flags & 4) && (mt.flags & 8);
+        // slot 0 holds the CTA's first segment, which may have begun in an
+        // earlier CTA; slot 1 its last, which may end in a later one
+        float* part = p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + (ordinal == 0 ? 0 : 1)) * PF;
+        finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, complete, part, merge, tid);
+        named_bar_sync(1, NW * 32);
+        ++ordinal;
       }
     }
   } else {
-    // ------------------------------------------------------------ consumers
+    // ------------------------------------------------------------ consumers (fp32)
     const int hw = lane >> 4, sub = lane & 15;
     const int rowbase = (warp * 2 + hw) * KPH;
     // Per key, the half-warp forms 2 HPW partial dot products per lane (s for
@@ -364,7 +633,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     float2 qf[HPW][H2], rf[HPW][H2], oa[HPW][H2], ua[HPW][H2];
     // running max of this lane's head, and l (score lanes) or z (probe lanes)
     float m_run = -INFINITY, lz = 0.f;
-    int ordinal = 0;
+    int ordinal = 0;  // segments finalised so far by this CTA
 #pragma unroll
     for (int g = 0; g < HPW; ++g) {
 #pragma unroll
@@ -508,7 +777,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (lane == 0) mbar_arrive(&empty[stage]);
 
       if (mt.flags & 2) {
-        // ---- finalise the segment: merge the 16 half-warp states
+        // ---- merge the two half-warp states, to shared memory
         float m[HPW], l[HPW], z[HPW];
 #pragma unroll
         for (int g = 0; g < HPW; ++g) {
@@ -553,59 +822,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
           }
         }
-        named_bar_sync(1, kDecConsumerWarps * 32);
+        named_bar_sync(1, NW * 32);
         const bool complete = (mt.flags & 4) && (mt.flags & 8);
-        const int slot = ordinal == 0 ? 0 : 1;
-        float* part = p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + slot) * PF;
-        for (int pr = tid; pr < HPW * D; pr += kDecConsumerWarps * 32) {
-          const int g = pr / D, c = pr % D;
-          float M = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, merge[(w * HPW + g) * PHF]);
-          float L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
-#pragma unroll
-          for (int w = 0; w < kDecConsumerWarps; ++w) {
-            const float* src = merge + (w * HPW + g) * PHF;
-            const float wt = merge_weight(src[0], M);
-            L += wt * src[1];
-            Z += wt * src[2];
-            O += wt * src[4 + c];
-            U += wt * src[4 + D + c];
-          }
-          if (MODE == kDecState && complete) {
-            float* sr = p.state + ((size_t)mt.b * p.Hq + h0 + g) * PHF;
-            if (c == 0) {
-              sr[0] = M;
-              sr[1] = L;
-              sr[2] = Z;
-              sr[3] = 0.f;
-            }
-            sr[4 + c] = O;
-            sr[4 + D + c] = U;
-          } else if (complete) {
-            // out = (1 + tbar) o - u with tbar = Z/L, o = O/L, u = U/L
-            const float inv = 1.f / L;
-            const float val = ((1.f + Z * inv) * O - U) * inv;
-            store_elem<T>(p.out, ((size_t)mt.b * p.Hq + h0 + g) * D + c, val);
-          } else {
-            float* ph = part + kPartHeader + g * PHF;
-            if (c == 0) {
-              ph[0] = M;
-              ph[1] = L;
-              ph[2] = Z;
-            }
-            ph[4 + c] = O;
-            ph[4 + D + c] = U;
-          }
-        }
-        if (!complete && tid == 0) {
-          int* hdr = reinterpret_cast<int*>(part);
-          hdr[1] = (mt.flags & 4) ? 1 : 0;
-          hdr[2] = (mt.flags & 8) ? 1 : 0;
-          hdr[3] = 0;
-          hdr[0] = mt.seg;
-        }
-        named_bar_sync(1, kDecConsumerWarps * 32);
+        float* part = p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + (ordinal == 0 ? 0 : 1)) * PF;
+        finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, complete, part, merge, tid);
+        named_bar_sync(1, NW * 32);
         ++ordinal;
       }
     }
@@ -750,20 +971,24 @@ constexpr int decode_smem_bytes(int hpw) {
   using Cfg = DecodeTile<T, D>;
   return 1024 + Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::STAGES * (int)sizeof(TileMeta) +
          2 * Cfg::STAGES * 8 + (int)sizeof(RangeInfo) + 20 * 8 +
-         kDecConsumerWarps * hpw * part_head_floats<D>() * 4 + 16 +
-         (2 * kDecConsumerWarps * kDecRedRegion + 2 * kDecConsumerWarps * 16) * 4;
+         Cfg::NW * hpw * part_head_floats<D>() * 4 + 16 +
+         (Cfg::MMA ? 0 : (2 * Cfg::NW * kDecRedRegion + 2 * Cfg::NW * 16) * 4);
 }
+static_assert(decode_smem_bytes<__nv_bfloat16, 128>(2) <= 227 * 1024, "shared memory");
+static_assert(decode_smem_bytes<__nv_bfloat16, 64>(2) <= 227 * 1024, "shared memory");
+static_assert(decode_smem_bytes<float, 128>(2) <= 227 * 1024, "shared memory");
+static_assert(decode_smem_bytes<float, 64>(2) <= 227 * 1024, "shared memory");
 
 template <typename T, int D, int HPW>
-cudaError_t launch_decode_t(const CUtensorMap& kmap, const CUtensorMap& vmap,
-                            const DecodeParams& p, cudaStream_t stream) {
+cudaError_t launch_decode_t(const DecodeMaps& m, const DecodeParams& p, cudaStream_t stream) {
+  using Cfg = DecodeTile<T, D>;
   const int smem = decode_smem_bytes<T, D>(HPW);
   auto kern = p.block_table ? plx_decode_splitk_kernel<T, D, HPW, kDecPaged>
                : p.state     ? plx_decode_splitk_kernel<T, D, HPW, kDecState>
                              : plx_decode_splitk_kernel<T, D, HPW, kDecContiguous>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<p.grid, kDecThreads, smem, stream>>>(kmap, vmap, p);
+  kern<<<p.grid, Cfg::THREADS, smem, stream>>>(m.k, m.v, m.k_chunk, m.v_chunk, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // The combine kernel is a programmatic dependent of the main kernel, so its
@@ -784,11 +1009,11 @@ cudaError_t launch_decode_t(const CUtensorMap& kmap, const CUtensorMap& vmap,
 }
 
 template <typename T, int D>
-cudaError_t launch_decode_d(const CUtensorMap& kmap, const CUtensorMap& vmap,
-                            const DecodeParams& p, int hpw, cudaStream_t stream) {
+cudaError_t launch_decode_d(const DecodeMaps& m, const DecodeParams& p, int hpw,
+                            cudaStream_t stream) {
   switch (hpw) {
-    case 1: return launch_decode_t<T, D, 1>(kmap, vmap, p, stream);
-    case 2: return launch_decode_t<T, D, 2>(kmap, vmap, p, stream);
+    case 1: return launch_decode_t<T, D, 1>(m, p, stream);
+    case 2: return launch_decode_t<T, D, 2>(m, p, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -832,14 +1057,14 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(bool bf16, int d, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                          const DecodeParams& p, int hpw, cudaStream_t stream) {
+cudaError_t launch_decode(bool bf16, int d, const DecodeMaps& m, const DecodeParams& p, int hpw,
+                          cudaStream_t stream) {
   if (bf16) {
-    if (d == 64) return launch_decode_d<__nv_bfloat16, 64>(kmap, vmap, p, hpw, stream);
-    if (d == 128) return launch_decode_d<__nv_bfloat16, 128>(kmap, vmap, p, hpw, stream);
+    if (d == 64) return launch_decode_d<__nv_bfloat16, 64>(m, p, hpw, stream);
+    if (d == 128) return launch_decode_d<__nv_bfloat16, 128>(m, p, hpw, stream);
   } else {
-    if (d == 64) return launch_decode_d<float, 64>(kmap, vmap, p, hpw, stream);
-    if (d == 128) return launch_decode_d<float, 128>(kmap, vmap, p, hpw, stream);
+    if (d == 64) return launch_decode_d<float, 64>(m, p, hpw, stream);
+    if (d == 128) return launch_decode_d<float, 128>(m, p, hpw, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -848,5 +1073,7 @@ int decode_tile_keys(bool bf16, int d) {
   (void)d;
   return bf16 ? DecodeTile<__nv_bfloat16, 128>::TK : DecodeTile<float, 128>::TK;
 }
+
+int decode_box_cols(bool bf16, int d) { return bf16 ? 64 : d; }
 
 }  // namespace plx

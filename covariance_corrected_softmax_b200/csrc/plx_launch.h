@@ -42,9 +42,17 @@ struct PrefillTcArgs {
 cudaError_t launch_prefill_simt(const PrefillSimtParams& p, int d, cudaStream_t stream);
 // Tensor-core (tcgen05) bf16 prefill; encodes its own TMA descriptors.
 cudaError_t launch_prefill_tc(const PrefillTcArgs& a, cudaStream_t stream);
-cudaError_t launch_decode(bool bf16, int d, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                          const DecodeParams& p, int hpw, cudaStream_t stream);
+// TMA maps of one decode call: k, v with tile-high boxes over the contiguous
+// cache; k_chunk, v_chunk with 16-row boxes over the contiguous cache (a
+// segment's partial last tile) or over the page pools (paged caches).  Boxes
+// are decode_box_cols() wide; bf16 boxes use the 128-byte swizzle.
+struct DecodeMaps {
+  CUtensorMap k, v, k_chunk, v_chunk;
+};
+cudaError_t launch_decode(bool bf16, int d, const DecodeMaps& m, const DecodeParams& p, int hpw,
+                          cudaStream_t stream);
 int decode_tile_keys(bool bf16, int d);
+int decode_box_cols(bool bf16, int d);
 // out[row] from R softmax states [R, rows, 2d + 4] (see DecodeParams::state).
 cudaError_t launch_merge_states(const float* states, int R, long long rows, void* out, int d,
                                 bool bf16, cudaStream_t stream);
@@ -53,6 +61,19 @@ cudaError_t launch_merge_states(const float* states, int R, long long rows, void
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
                              const int32_t* seqlens, int B, int Hkv, int d, int elem_bytes,
                              int S_max, cudaStream_t stream);
+
+// rho[M, N] = x[M, K] w[N, K]^T (the probe projection): bf16 on the tensor
+// cores (K % 8 == 0, N % 8 == 0, 16-byte aligned rows), fp32 on CUDA cores.
+cudaError_t launch_probe_projection(const void* x, const void* w, void* rho, int M, int N, int K,
+                                    bool bf16, int num_sms, unsigned* err, cudaStream_t stream);
+
+// Gradients of the prefill operator (CUDA cores): dq, drho [B, L, Hq, d],
+// dk, dv [B, L, Hkv, d], all fp32; workspace of prefill_bwd_workspace_bytes().
+size_t prefill_bwd_workspace_bytes(int B, int L, int Hq);
+cudaError_t launch_prefill_bwd(const void* q, const void* rho, const void* k, const void* v,
+                               const void* dout, float* dq, float* drho, float* dk, float* dv,
+                               void* workspace, int causal, int B, int L, int Hq, int Hkv, int d,
+                               bool bf16, float scale, cudaStream_t stream);
 
 // One warp that waits on an mbarrier nothing ever completes, with the
 // device's bounded wait: it records kDevTimeoutMbarrier when the limit runs out

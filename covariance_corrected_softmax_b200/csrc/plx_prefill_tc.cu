@@ -16,8 +16,8 @@
 //               keys into a 4-stage ring (128-byte swizzled, UMMA-canonical).
 //   warp 1      S/T issuer (one thread): S = Q K^T and T = R K^T of each key
 //               tile (sharing the K tile).
-//   warp 2      converts each V tile to fp16 in place; also allocates and
-//               frees the TMEM columns.
+//   warps 2, 12 convert each V tile to fp16 in place (half a tile each);
+//               warp 2 also allocates and frees the TMEM columns.
 //   warp 3      PV issuer (one thread): O += P V and U += (P o T) V of each
 //               key tile (sharing the V tile).
 //   warps 4-11  softmax + epilogue: two warpgroups; thread (row, half) owns
@@ -48,8 +48,17 @@
 // grows only if |t| would push it past fp16's range; O and U (with their l, z
 // columns) pass through registers only when either changes, after P and P t
 // of the tile are stored.
-// Range: |v| and |rho . k| must stay below 65504 (fp16); a non-finite result
-// is reported through the device error word.
+// Range: V enters the fp16 products as a block floating-point value: the
+// converter warp finds the largest |v| of each V tile and scales the tile by
+// 2^-E before rounding it to fp16, E being the running maximum, over the
+// unit's tiles so far, of floor(log2 max|v|) - 14 (so every scaled value is
+// below 2^15).  When E grows, the V columns of O and U are rescaled with the
+// other lazy rescales; the epilogue multiplies by 2^E.  The ones block is not
+// scaled, so l and z are unaffected.  Any finite bf16 V thus keeps fp16's 11
+// significant bits relative to the largest |v| of its tile.  P t carries its
+// own power-of-two scale (eu, above).  A non-finite result (inputs whose result
+// exceeds fp32, or non-finite inputs) is reported through the device error
+// word.
 #include "plx_launch.h"
 
 namespace plx {
@@ -61,14 +70,24 @@ constexpr int kBN = 64;       // keys per tile
 constexpr int kHalf = kBN / 2;  // key columns per softmax thread
 constexpr int kStages = 4;    // K/V ring depth (the shared-memory layout below assumes 4)
 constexpr int kSoftWarps = 8;   // two softmax warpgroups
-constexpr int kConvWarps = 1;   // V converter
-constexpr int kThreads = (4 + kSoftWarps) * 32;
+constexpr int kConvWarps = 2;   // V converters: warp 2 and the last warp
+constexpr int kThreads = (4 + kSoftWarps + 1) * 32;
+constexpr int kConvWarp2 = 4 + kSoftWarps;  // the second converter's warp index
 // Lazy rescaling: the running max m moves only when a score exceeds it by more
 // than 2^kRescaleBits, so P <= 2^kRescaleBits; |t| 2^-eu is kept below
 // 2^kTBits so that |P t 2^-eu| < 2^15 stays inside fp16's range.
 constexpr int kRescaleBits = 8;
 constexpr int kTBits = 15 - kRescaleBits;
 constexpr uint32_t kOnesBytes = 8192;      // 64 keys x 64 fp16 ones, 128-byte rows
+// Block exponent E of V (see the header comment): clamped to [kVExpMin,
+// kVExpMax] so that 2^-E and 2^E stay normal fp32 numbers.  A tile whose
+// largest |v| lies in [2^kVLowBits, 2^(kVHeadroomBits + 1)) is kept as it is
+// (E = 0): fp16 holds it and every value down to 2^-8 of the largest with full
+// precision, and the conversion needs no multiply.
+constexpr int kVExpMin = -100;
+constexpr int kVExpMax = 113;
+constexpr int kVHeadroomBits = 14;   // scaled |v| < 2^(kVHeadroomBits + 1)
+constexpr int kVLowBits = -6;
 // Key pairs (of a thread's 16) whose 2^x runs on the FMA pipe (exp2_poly2)
 // rather than the special-function unit, which also does the fp16 packing.
 constexpr uint32_t kPolyPairs = 0x8888u;
@@ -202,12 +221,15 @@ struct Bars {
   uint64_t s_free;             // S, T of tile t copied to registers (softmax warps)
   uint64_t p_full;             // P, P t of tile t stored (softmax warps)
   uint64_t o_done;             // PV of tile t completed
+  uint64_t conv_sync;          // both converters posted their tile's max |v|
+  int vexp[kStages];           // block exponent E the stage's V was scaled by
 };
 
 // Shared memory the two halves of a row exchange through (two slots, used
 // alternately, so one named barrier per exchange suffices).
 struct Xchg {
   float2 tile[2][2][kBM];   // [slot][half][row]: (partial max, partial max |t|)
+  uint32_t vmax[2][2];      // [tile parity][converter]: partial max |v| (bf16 bits)
 };
 
 template <int D, typename OutT, bool VARLEN>
@@ -244,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->s_free, kSoftWarps);  // one arrival per softmax warp
     mbar_init(&bars->p_full, kSoftWarps);
     mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->conv_sync, kConvWarps);
     fence_mbarrier_init();
   }
   {
@@ -415,41 +438,90 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bars->drain, 0, &never, p.err);
     }
     __syncwarp();
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ V converter
-    // V of each tile -> fp16 in place (the PV products run in fp16), eight
-    // 16-byte words per thread at a time.
+  } else if (warp == 2 || warp == kConvWarp2) {
+    // ------------------------------------------------------------ V converters
+    // V of each tile -> fp16 in place (the PV products run in fp16), scaled by
+    // 2^-E (block floating point, E the unit's running block exponent).  Each
+    // of the two converter warps takes half of the tile's 16-byte words: a
+    // first pass finds its half's largest |v| (bf16 magnitudes, packed max),
+    // the halves are combined through shared memory, a second pass scales (if
+    // E != 0) and converts, eight words per thread at a time.
+    constexpr int kWords = C::KV_BYTES / 16;         // 16-byte words of a V tile
+    constexpr int kIters = kWords / (2 * 32 * 8);    // per converter, 8 words per step
+    static_assert(kIters >= 1 && kWords % (2 * 32 * 8) == 0, "converter split");
+    const int cw = warp == 2 ? 0 : 1;                // which half of the words
     int g = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
       const int n = unit_of<VARLEN>(p, u).n;
+      int ve = kVExpMin;
       for (int j = 0; j < n; ++j) {
         const int t = g + j, st = t % kStages;
         if (!mbar_wait(&bars->kv_full[st], (t / kStages) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
+        // word w of the tile: column block w / 512, word w % 512 of it
+        auto word = [&](int h, int q) {
+          const int w = (cw * kIters + h) * 256 + 32 * q + lane;
+          return reinterpret_cast<uint4*>(sKV + C::v_box(st, w >> 9)) + (w & 511);
+        };
+        uint32_t mx = 0;
 #pragma unroll 1
-        for (int h = 0; h < C::KV_BYTES / (16 * 32 * 8); ++h) {
-          // column block h / 2, its 256-word half h % 2
-          uint4* vt = reinterpret_cast<uint4*>(sKV + C::v_box(st, h >> 1)) + (h & 1) * 256 + lane;
-          uint4 w[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) w[q] = vt[32 * q];
+        for (int h = 0; h < kIters; ++h) {
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            float2 f;
-            f = bf16x2_to_float2(w[q].x);
-            w[q].x = float2_to_f16x2(f.x, f.y);
-            f = bf16x2_to_float2(w[q].y);
-            w[q].y = float2_to_f16x2(f.x, f.y);
-            f = bf16x2_to_float2(w[q].z);
-            w[q].z = float2_to_f16x2(f.x, f.y);
-            f = bf16x2_to_float2(w[q].w);
-            w[q].w = float2_to_f16x2(f.x, f.y);
-            vt[32 * q] = w[q];
+            const uint4 w = *word(h, q);
+            mx = bf16x2_max(mx, bf16x2_max(bf16x2_max(w.x & 0x7fff7fffu, w.y & 0x7fff7fffu),
+                                           bf16x2_max(w.z & 0x7fff7fffu, w.w & 0x7fff7fffu)));
           }
         }
+        mx = __reduce_max_sync(0xffffffffu, max(mx & 0xffffu, mx >> 16));
+        // combine with the other converter's half (slots alternate by tile,
+        // so one arrival per tile and converter suffices)
+        if (lane == 0) {
+          xch->vmax[t & 1][cw] = mx;
+          mbar_arrive(&bars->conv_sync);
+        }
+        if (!mbar_wait(&bars->conv_sync, t & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        mx = max(xch->vmax[t & 1][0], xch->vmax[t & 1][1]);
+        if (mx != 0) {
+          // floor(log2 |v|max) from the bf16 exponent field (subnormals count as
+          // 2^-127, inf and NaN as 2^128: those results are reported anyway)
+          const int fl = (int)(mx >> 7) - 127;
+          const int e = (fl >= kVLowBits && fl <= kVHeadroomBits)
+                            ? 0
+                            : min(kVExpMax, max(kVExpMin, fl - kVHeadroomBits));
+          ve = max(ve, e);
+        }
+        const int vuse = max(ve, kVExpMin);
+        const float sc = __int_as_float((127 - vuse) << 23);  // 2^-E, exact
+        const float2 sc2 = make_float2(sc, sc);
+        const bool scaled = vuse != 0;
+#pragma unroll 1
+        for (int h = 0; h < kIters; ++h) {
+          uint4 w[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) w[q] = *word(h, q);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float2 f0 = bf16x2_to_float2(w[q].x), f1 = bf16x2_to_float2(w[q].y);
+            float2 f2v = bf16x2_to_float2(w[q].z), f3 = bf16x2_to_float2(w[q].w);
+            if (scaled) {
+              f0 = __fmul2_rn(f0, sc2);
+              f1 = __fmul2_rn(f1, sc2);
+              f2v = __fmul2_rn(f2v, sc2);
+              f3 = __fmul2_rn(f3, sc2);
+            }
+            w[q] = make_uint4(float2_to_f16x2(f0.x, f0.y), float2_to_f16x2(f1.x, f1.y),
+                              float2_to_f16x2(f2v.x, f2v.y), float2_to_f16x2(f3.x, f3.y));
+            *word(h, q) = w[q];
+          }
+        }
+        if (cw == 0 && lane == 0) bars->vexp[st] = vuse;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->v_ready[st]);
@@ -476,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (lazy rescaling).  eu (>= 0) keeps P t 2^-eu in fp16's range.
       float m_run = -INFINITY;
       int eu = 0;
+      int ve = 0;  // block exponent of the V columns of O and U (see the converter)
       float tlim = (float)(1 << kTBits), tsc = 1.f;  // 2^(kTBits + eu), 2^-eu
       for (int j = 0; j < x.n; ++j) {
         const int t = g + j;
@@ -536,10 +609,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         int eu_new = eu;
         if (tmax >= tlim) eu_new = max(eu, (int)ceilf(log2f(tmax)) - (kTBits - 1));
         const bool ubump = eu_new > eu;
+        // the block exponent the converter scaled this tile's V by
+        const int st = t % kStages;
+        if (!mbar_wait(&bars->v_ready[st], (t / kStages) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        const int ve_new = bars->vexp[st];
+        const bool vchange = j > 0 && ve_new != ve;  // the same for every thread of the CTA
+        float vf = 1.f;  // factor of the V columns of O and U (not of l, z)
+        if (vchange) vf = exp2f((float)(ve - ve_new));
+        ve = ve_new;
         // O and U (with l, z) are rescaled below, after P and P t are stored;
         // P and P t already use the new m and eu.  (The partner warp holds the
         // same rows, so both warps of a row take the branch together.)
-        const bool rescale = __any_sync(0xffffffffu, resc || ubump);
+        const bool rescale = __any_sync(0xffffffffu, resc || ubump) || vchange;
         float fr = 1.f;  // this half's factor: half 0 rescales O (and l), half 1 U (and z)
         if (rescale) {
           const float alpha = resc ? exp2f(m_run - m_new) : 1.f;
@@ -601,14 +685,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st16(lane_addr + C::COL_PT + my_cols / 2, pk);
         if (rescale) {
           const uint32_t base = lane_addr + (half == 0 ? C::COL_O : C::COL_U);
+          const float frv = fr * vf;  // the V columns; the ones columns take fr
 #pragma unroll 1
           for (int cc = 0; cc < D; cc += 64) {
             uint32_t wa[32], wb[32];
             tmem_ld2x32_sync(base + cc, base + cc + 32, wa, wb);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              wa[e] = __float_as_uint(__uint_as_float(wa[e]) * fr);
-              wb[e] = __float_as_uint(__uint_as_float(wb[e]) * fr);
+              wa[e] = __float_as_uint(__uint_as_float(wa[e]) * frv);
+              wb[e] = __float_as_uint(__uint_as_float(wb[e]) * frv);
             }
             tmem_st32(base + cc, wa);
             tmem_st32(base + cc + 32, wb);
@@ -635,8 +720,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float l = __uint_as_float(lw), z = __uint_as_float(zw);
       const float inv = 1.f / l;
       const float usc = exp2f((float)eu);           // undo the P t scaling
-      const float c1 = (1.f + z * usc * inv) * inv;
-      const float cu = usc * inv;
+      const float vsc = exp2f((float)ve);           // and the block scaling of V
+      const float c1 = (1.f + z * usc * inv) * inv * vsc;
+      const float cu = usc * inv * vsc;
       OutT* orow = static_cast<OutT*>(p.out) + (((size_t)x.tok0 + i) * p.Hq + x.h) * D;
 #pragma unroll 1
       for (int cc = half * (D / 2); cc < (half + 1) * (D / 2); cc += 32) {

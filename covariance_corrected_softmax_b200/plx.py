@@ -68,6 +68,16 @@ def lib() -> ctypes.CDLL:
         L.plx_last_cuda_error.restype = i
         L.plx_device_error.argtypes = [ctypes.POINTER(i), i]
         L.plx_device_error.restype = i
+        L.plx_probe_projection.argtypes = [vp, vp, vp, i, i, i, i, vp]
+        L.plx_probe_projection.restype = i
+        L.plx_prefill_fwd_x.argtypes = [vp] * 8 + [i] * 8 + [f, vp]
+        L.plx_prefill_fwd_x.restype = i
+        L.plx_decode_x.argtypes = [vp] * 8 + [i] * 7 + [f, vp, sz, vp]
+        L.plx_decode_x.restype = i
+        L.plx_prefill_bwd_workspace_bytes.argtypes = [i, i, i]
+        L.plx_prefill_bwd_workspace_bytes.restype = sz
+        L.plx_prefill_bwd.argtypes = [vp] * 9 + [i] * 7 + [f, vp, sz, vp]
+        L.plx_prefill_bwd.restype = i
         L.plx_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.plx_set_wait_limit_ns.restype = i
         L.plx_selftest_wait.argtypes = [vp]
@@ -173,6 +183,100 @@ def prefill_varlen(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch
                                   _stream(stream))
     _check(st, "plx_prefill_varlen")
     return out, (lse if return_lse else None)
+
+
+def probe_projection(x: torch.Tensor, w_r: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """rho = x W_R^T: x [..., K], w_r [N, K] -> [..., N] in x's dtype."""
+    _same(x, w_r)
+    K = x.shape[-1]
+    N = w_r.shape[0]
+    if w_r.dim() != 2 or w_r.shape[1] != K:
+        raise ValueError("w_r must be [N, K] with K the last dimension of x")
+    M = x.numel() // K if K else 0
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=x.dtype, device=x.device)
+    st = lib().plx_probe_projection(_ptr(x), _ptr(w_r), _ptr(out), M, N, K, _dtype_code(x),
+                                    _stream(stream))
+    _check(st, "plx_probe_projection")
+    return out
+
+
+def prefill_x(q: torch.Tensor, x: torch.Tensor, w_r: torch.Tensor, k: torch.Tensor,
+              v: torch.Tensor, causal: bool = True, softmax_scale: Optional[float] = None,
+              return_lse: bool = True, stream=None
+              ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """Forward with rho = x W_R^T computed on the device: q [B, L, Hq, d];
+    x [B, L, d_model]; w_r [Hq d, d_model]; k, v [B, L, Hkv, d].  Returns
+    (out, rho, lse)."""
+    _same(q, x, w_r, k, v)
+    B, L, Hq, d = q.shape
+    Hkv, dm = k.shape[2], x.shape[-1]
+    if x.shape != (B, L, dm) or w_r.shape != (Hq * d, dm) or k.shape != (B, L, Hkv, d) or \
+            v.shape != k.shape:
+        raise ValueError("shape mismatch among q, x, w_r, k, v")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    rho = torch.empty_like(q)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device) if return_lse else None
+    st = lib().plx_prefill_fwd_x(_ptr(q), _ptr(x), _ptr(w_r), _ptr(k), _ptr(v), _ptr(rho),
+                                 _ptr(out), _ptr(lse), int(bool(causal)), B, L, Hq, Hkv, d, dm,
+                                 _dtype_code(q), scale, _stream(stream))
+    _check(st, "plx_prefill_fwd_x")
+    return out, rho, lse
+
+
+def decode_x(q: torch.Tensor, x: torch.Tensor, w_r: torch.Tensor, k_cache: torch.Tensor,
+             v_cache: torch.Tensor, seqlens: torch.Tensor, softmax_scale: Optional[float] = None,
+             workspace: Optional[torch.Tensor] = None, stream=None
+             ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Decode with rho = x W_R^T computed on the device: q [B, Hq, d];
+    x [B, d_model]; w_r [Hq d, d_model].  Returns (out, rho)."""
+    _same(q, x, w_r, k_cache, v_cache)
+    B, Hq, d = q.shape
+    S_max, Hkv = k_cache.shape[1], k_cache.shape[2]
+    dm = x.shape[-1]
+    if x.shape != (B, dm) or w_r.shape != (Hq * d, dm) or \
+            k_cache.shape != (B, S_max, Hkv, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch among q, x, w_r, k_cache, v_cache")
+    if seqlens.dtype != torch.int32 or seqlens.device != q.device or seqlens.numel() != B:
+        raise ValueError("seqlens must be int32 [B] on the same device")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    rho = torch.empty_like(q)
+    out = torch.empty_like(q)
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, Hkv, d, S_max, device=q.device)
+    st = lib().plx_decode_x(_ptr(q), _ptr(x), _ptr(w_r), _ptr(k_cache), _ptr(v_cache),
+                            _ptr(seqlens), _ptr(rho), _ptr(out), B, Hq, Hkv, d, S_max, dm,
+                            _dtype_code(q), scale, _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "plx_decode_x")
+    return out, rho
+
+
+def prefill_bwd(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                dout: torch.Tensor, causal: bool = True, softmax_scale: Optional[float] = None,
+                stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients (dq, drho, dk, dv), fp32, of sum(dout * out) for the forward
+    plx.prefill(q, rho, k, v, causal, softmax_scale)."""
+    _same(q, rho, k, v, dout)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if rho.shape != q.shape or dout.shape != q.shape or k.shape != (B, L, Hkv, d) or \
+            v.shape != k.shape:
+        raise ValueError("shape mismatch among q, rho, k, v, dout")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, drho = torch.empty(q.shape, **f32), torch.empty(q.shape, **f32)
+    dk, dv = torch.empty(k.shape, **f32), torch.empty(k.shape, **f32)
+    nws = int(lib().plx_prefill_bwd_workspace_bytes(B, L, Hq))
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=q.device)
+    st = lib().plx_prefill_bwd(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(dout),
+                               _ptr(dq), _ptr(drho), _ptr(dk), _ptr(dv), int(bool(causal)), B, L,
+                               Hq, Hkv, d, _dtype_code(q), scale, _ptr(ws), ws.numel(),
+                               _stream(stream))
+    _check(st, "plx_prefill_bwd")
+    return dq, drho, dk, dv
 
 
 def decode_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, S_max: int) -> int:

@@ -192,6 +192,18 @@ def make_decode(shape: DecodeShape, seed: int = 0, device="cpu",
     return out
 
 
+def make_probe_inputs(lead: Tuple[int, ...], d_model: int, n_out: int, seed: int = 0,
+                      device="cpu", dtype=torch.bfloat16, w_std: float = 0.02
+                      ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Layer inputs x [*lead, d_model] ~ N(0, 1) and a projection W_R
+    [n_out, d_model] ~ N(0, w_std^2) (the decode workload's probe recipe:
+    width 2048, std 0.02), rounded to dtype."""
+    g = _gen(device, seed)
+    x = _normal(tuple(lead) + (d_model,), 1.0, g, device, dtype)
+    w = _normal((n_out, d_model), w_std, g, device, dtype)
+    return x, w
+
+
 def sample_rows_prefill(shape: PrefillShape, n: int, seed: int = 1,
                         stratified: bool = True) -> np.ndarray:
     """n seeded (b, h, i) rows; with ``stratified`` row k lies in [kL/n, (k+1)L/n)."""

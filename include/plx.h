@@ -139,6 +139,73 @@ PLX_API plx_status plx_prefill_varlen(const void* q, const void* rho, const void
                                       float softmax_scale, void* stream);
 
 /*
+ * plx_probe_projection -- the probe projection rho = W_R x for a block of
+ * tokens (page 1 section 1.3: one extra projection matrix, rho_i = W_R x_i;
+ * page 3: the probe is computed from the layer input), as the GEMM
+ *
+ *     rho[M, N] = x[M, K] W_R[N, K]^T     (fp32 accumulation)
+ *
+ *   x    : [M, K]  layer inputs, one row per token (K = model width)
+ *   w_r  : [N, K]  W_R, row n = output feature n (N = H_q * d for the
+ *                  attention's probe layout [.., H_q, d])
+ *   rho  : [M, N]  written, in dtype
+ * PLX_BF16 runs on the tensor cores and needs K % 8 == 0 and N % 8 == 0
+ * (else PLX_ERR_UNSUPPORTED); PLX_F32 on the CUDA cores.  M == 0 or N == 0 is
+ * a no-op; K >= 1.
+ */
+PLX_API plx_status plx_probe_projection(const void* x, const void* w_r, void* rho, int M, int N,
+                                        int K, plx_dtype dtype, void* stream);
+
+/*
+ * plx_prefill_fwd_x -- plx_prefill_fwd with the probes computed from the layer
+ * input: rho = x W_R^T (plx_probe_projection with M = B L, N = H_q d,
+ * K = d_model), then the attention forward, both on stream.
+ *
+ *   x   : [B, L, d_model]   w_r : [H_q d, d_model]
+ *   rho : [B, L, H_q, d] written (the probes; the backward needs them too)
+ * Every other argument as plx_prefill_fwd.  All arguments of both steps are
+ * checked before anything is enqueued.
+ */
+PLX_API plx_status plx_prefill_fwd_x(const void* q, const void* x, const void* w_r,
+                                     const void* k, const void* v, void* rho, void* out,
+                                     float* lse, int causal, int B, int L, int H_q, int H_kv,
+                                     int d, int d_model, plx_dtype dtype, float softmax_scale,
+                                     void* stream);
+
+/*
+ * plx_prefill_bwd -- gradients of the prefill operator, for training (page 1
+ * section 2.3 trains W_R with the rest of the model; the pages print no
+ * gradient, so it is derived from the operator of section 1.3):
+ *
+ *   with g = dLoss/dout, row i, keys j, a_j = softmax_j(scale q.k_j),
+ *   t_j = rho.k_j, tbar = sum a t, o = sum a v, c_j = 1 + tbar - t_j:
+ *     dv_j += a_j c_j g
+ *     dt_j  = a_j (g.o - g.v_j)
+ *     ds_j  = a_j (c_j g.v_j + t_j g.o - g.out - tbar g.o)
+ *     dq   += scale sum_j ds_j k_j,   drho += sum_j dt_j k_j,
+ *     dk_j += scale ds_j q + dt_j rho
+ *
+ *   q, rho, dout : [B, L, H_q, d] in dtype      k, v : [B, L, H_kv, d]
+ *   dq, drho     : [B, L, H_q, d] fp32, written
+ *   dk, dv       : [B, L, H_kv, d] fp32, written (summed over the query
+ *                  heads that share a KV head)
+ *   workspace    : plx_prefill_bwd_workspace_bytes(B, L, H_q) bytes, 16-byte
+ *                  aligned, no initialisation needed
+ * Other arguments as plx_prefill_fwd.  Neither the forward's output nor its
+ * lse is needed: the kernels recompute what they use, the softmax normaliser
+ * included, from q, rho, k, v in fp32 (where one key dominates a row, the
+ * gradient's a (X - D) terms cancel and would amplify the fp16 rounding that
+ * the tensor-core forward's normaliser carries).  Runs on the CUDA cores with
+ * fp32 arithmetic (a correctness path, not tuned).
+ */
+PLX_API size_t plx_prefill_bwd_workspace_bytes(int B, int L, int H_q);
+PLX_API plx_status plx_prefill_bwd(const void* q, const void* rho, const void* k, const void* v,
+                                   const void* dout, float* dq, float* drho, float* dk,
+                                   float* dv, int causal, int B, int L, int H_q, int H_kv, int d,
+                                   plx_dtype dtype, float softmax_scale, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
  * plx_decode_workspace_bytes -- device workspace that plx_decode needs for the
  * given shape on the CURRENT device (it depends on the device's SM count).
  * Returns 0 for an invalid shape.
@@ -165,6 +232,22 @@ PLX_API plx_status plx_decode(const void* q, const void* rho, const void* k_cach
                       const void* v_cache, const int32_t* seqlens, void* out, int B, int H_q,
                       int H_kv, int d, int S_max, plx_dtype dtype, float softmax_scale,
                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * plx_decode_x -- plx_decode with the new token's probes computed from its
+ * layer input: rho = x W_R^T (plx_probe_projection with M = B, N = H_q d,
+ * K = d_model), then the decode, both on stream.
+ *
+ *   x   : [B, d_model]   w_r : [H_q d, d_model]
+ *   rho : [B, H_q, d] written
+ * Every other argument, the workspace rule and the errors as plx_decode.  All
+ * arguments of both steps are checked before anything is enqueued.
+ */
+PLX_API plx_status plx_decode_x(const void* q, const void* x, const void* w_r,
+                                const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                                void* rho, void* out, int B, int H_q, int H_kv, int d, int S_max,
+                                int d_model, plx_dtype dtype, float softmax_scale,
+                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * plx_decode_state -- plx_decode, but instead of out it writes each (b, h)

@@ -232,3 +232,61 @@ def test_wait_limit_rejects_out_of_range_values():
     L = plx.lib()
     assert L.plx_set_wait_limit_ns(999) == INV
     assert L.plx_set_wait_limit_ns(61 * 10 ** 9) == INV
+
+
+def test_probe_projection_rejects():
+    L = plx.lib()
+    f = L.plx_probe_projection
+    assert f(FAKE, FAKE, FAKE, 4, 16, 8, 7, None) == INV             # dtype
+    assert f(FAKE, FAKE, FAKE, -1, 16, 8, plx.PLX_BF16, None) == INV  # M
+    assert f(FAKE, FAKE, FAKE, 4, 16, 0, plx.PLX_BF16, None) == INV   # K
+    assert f(None, FAKE, FAKE, 4, 16, 8, plx.PLX_BF16, None) == INV
+    assert f(FAKE, FAKE + 8, FAKE, 4, 16, 8, plx.PLX_BF16, None) == INV
+    assert f(FAKE, FAKE, FAKE, 4, 16, 12, plx.PLX_BF16, None) == plx.PLX_ERR_UNSUPPORTED  # K % 8
+    assert f(FAKE, FAKE, FAKE, 4, 20, 8, plx.PLX_BF16, None) == plx.PLX_ERR_UNSUPPORTED  # N % 8
+    assert f(None, None, None, 0, 16, 8, plx.PLX_BF16, None) == plx.PLX_OK  # M = 0: no-op
+
+
+def test_prefill_x_and_decode_x_check_both_steps_first():
+    L = plx.lib()
+    # bad attention argument (d = 96) with a valid projection: nothing launched
+    assert L.plx_prefill_fwd_x(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 2, 1,
+                               96, 64, plx.PLX_BF16, 1.0, None) == INV
+    # bad projection (x misaligned) with valid attention arguments
+    assert L.plx_prefill_fwd_x(FAKE, FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 2,
+                               1, 64, 64, plx.PLX_BF16, 1.0, None) == INV
+    assert L.plx_prefill_fwd_x(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 2, 1,
+                               64, 0, plx.PLX_BF16, 1.0, None) == INV  # d_model
+    assert L.plx_decode_x(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, FAKE, FAKE, 2, 4, 2, 128, 64,
+                          256, plx.PLX_BF16, 1.0, FAKE, 1 << 20, None) == INV  # seqlens
+    assert L.plx_decode_x(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 2, 128, 64,
+                          255, plx.PLX_BF16, 1.0, FAKE, 1 << 20, None) == plx.PLX_ERR_UNSUPPORTED
+    assert L.plx_decode_x(None, None, None, None, None, None, None, None, 0, 4, 2, 128, 64,
+                          256, plx.PLX_BF16, 1.0, None, 0, None) == plx.PLX_OK
+
+
+def _bwd(**kw):
+    a = dict(q=FAKE, rho=FAKE, k=FAKE, v=FAKE, g=FAKE, dq=FAKE, dr=FAKE, dk=FAKE,
+             dv=FAKE, causal=1, B=1, L=16, Hq=2, Hkv=1, d=64, dtype=plx.PLX_BF16, scale=0.1,
+             ws=FAKE, wsb=1 << 20)
+    a.update(kw)
+    return plx.lib().plx_prefill_bwd(a["q"], a["rho"], a["k"], a["v"], a["g"], a["dq"],
+                                     a["dr"], a["dk"], a["dv"], a["causal"], a["B"], a["L"],
+                                     a["Hq"], a["Hkv"], a["d"], a["dtype"], a["scale"], a["ws"],
+                                     a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(d=96), dict(Hq=3, Hkv=2), dict(causal=2), dict(L=-1), dict(dtype=5),
+    dict(scale=float("nan")), dict(q=None), dict(g=None), dict(dk=None), dict(ws=None),
+    dict(dv=FAKE + 8), dict(g=FAKE + 4),
+])
+def test_prefill_bwd_rejects(kw):
+    assert _bwd(**kw) == INV
+
+
+def test_prefill_bwd_workspace():
+    L = plx.lib()
+    assert L.plx_prefill_bwd_workspace_bytes(2, 100, 4) == 2 * 100 * 4 * 16
+    assert _bwd(wsb=16 * 2 * 16 - 1) == plx.PLX_ERR_WORKSPACE_TOO_SMALL
+    assert _bwd(B=0, q=None) == plx.PLX_OK
