@@ -363,7 +363,7 @@ def bench_prefill(plx, W, shape, steps, warmup, world, device, rank):
 
 
 # ------------------------------------------------------------------ decode grid
-def bench_decode_sweep(plx, W, peaks, device, max_cells=None):
+def bench_decode_sweep(plx, W, peaks, device, only=None):
     """Every cell of the decode grid (batch x context, ragged lengths U[ctx/2,
     ctx], caches capped under 120e9 bytes).  Each call is timed alone with CUDA
     events, after a 256 MiB buffer (twice the L2) has been written, so every
@@ -372,7 +372,9 @@ def bench_decode_sweep(plx, W, peaks, device, max_cells=None):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
     cells = []
-    for cell in W.sweep_cells()[:max_cells]:
+    for cell in W.sweep_cells():
+        if only and f"{cell.B}x{cell.ctx}" not in only:
+            continue
         inp = W.make_decode(cell, seed=0, device=device)
         ws = plx.decode_workspace(cell.B, cell.Hq, cell.Hkv, cell.d, cell.S_max, device=device)
         out = torch.empty_like(inp["q"])
@@ -504,6 +506,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-I/O leg (profiling)")
     ap.add_argument("--no-sweep", action="store_true", help="skip the decode grid")
+    ap.add_argument("--sweep-cells", nargs="*", default=None,
+                    help="run only these grid cells, as BATCHxCONTEXT (e.g. 64x32768)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -556,7 +560,7 @@ def main():
     sweep = None
     if not args.no_sweep:
         with ClockSampler(gpu_index()) as clk:
-            cells = bench_decode_sweep(plx, W, peaks, device)
+            cells = bench_decode_sweep(plx, W, peaks, device, args.sweep_cells)
         long_ctx = [c for c in cells if c["context"] >= 8192 and not c["launch_bound"]]
         sweep = {"grid": "H_q=16, H_kv=8, d=128, bf16; batch x context, lengths U[ctx/2, ctx]",
                  "timing": "median of per-call CUDA-event times, 256 MiB L2 flush before each call",

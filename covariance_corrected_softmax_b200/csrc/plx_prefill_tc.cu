@@ -177,6 +177,36 @@ struct Unit {
 };
 
 template <bool VARLEN>
+__device__ __forceinline__ Unit unit_of(const TcParams& p, int u);
+
+// The units the recomputing instance (SAFE) takes: a bit per unit of this CTA
+// (u = blockIdx.x + k gridDim.x), set where the fast instance left the marker.
+constexpr int kMaskUnits = 16384;   // units per CTA the mask covers (2 KB)
+
+// Marker a unit of the fast instance leaves in column 0 of its first row when
+// its V lies outside the range fp16 holds as it is (a NaN no arithmetic makes).
+constexpr uint16_t kMarkBf16 = 0x7FABu;
+constexpr uint32_t kMarkF32 = 0x7FABCDEFu;
+
+template <typename OutT>
+__device__ __forceinline__ bool is_marked(const void* out, size_t idx) {
+  if constexpr (sizeof(OutT) == 2)
+    return reinterpret_cast<const volatile uint16_t*>(out)[idx] == kMarkBf16;
+  else
+    return reinterpret_cast<const volatile uint32_t*>(out)[idx] == kMarkF32;
+}
+
+template <bool VARLEN, bool SAFE>
+__device__ __forceinline__ Unit unit_at(const TcParams& p, int u, const uint32_t* mask) {
+  Unit x = unit_of<VARLEN>(p, u);
+  if constexpr (SAFE) {
+    const int k = (u - (int)blockIdx.x) / (int)gridDim.x;
+    if (!((mask[k >> 5] >> (k & 31)) & 1u)) x.n = 0;
+  }
+  return x;
+}
+
+template <bool VARLEN>
 __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
   Unit x;
   const int bh = p.B * p.Hq;
@@ -221,18 +251,58 @@ struct Bars {
   uint64_t s_free;             // S, T of tile t copied to registers (softmax warps)
   uint64_t p_full;             // P, P t of tile t stored (softmax warps)
   uint64_t o_done;             // PV of tile t completed
-  uint64_t conv_sync;          // both converters posted their tile's max |v|
-  int vexp[kStages];           // block exponent E the stage's V was scaled by
+  uint64_t v_reload[2];        // a V column block fetched again (rare: its range changed E)
+  uint64_t v_rescaled;         // O, U rescaled for a changed E (softmax warps; rare)
+  int2 vtag[kStages][2];       // per column block: (tile number, exponent E it was scaled by)
+  int2 vunit[8][2];            // fast instance, per converter: (unit count, V out of range)
 };
 
 // Shared memory the two halves of a row exchange through (two slots, used
 // alternately, so one named barrier per exchange suffices).
 struct Xchg {
   float2 tile[2][2][kBM];   // [slot][half][row]: (partial max, partial max |t|)
-  uint32_t vmax[2][2];      // [tile parity][converter]: partial max |v| (bf16 bits)
 };
 
-template <int D, typename OutT, bool VARLEN>
+// Reads the block exponents E the converters scaled tile t's V column blocks
+// by (each posted with the tile number in one 8-byte word), waiting (bounded)
+// until both are posted.  Returns false on a timeout or an abort.
+template <int KB>
+__device__ __forceinline__ bool read_vtags(const int2 (*vtag)[2], int t, int (&e)[2],
+                                           volatile int* abort_flag, unsigned* err) {
+  const int st = t % kStages;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    e[b] = 0;
+    if (b >= KB) continue;
+    volatile const unsigned long long* tag =
+        reinterpret_cast<volatile const unsigned long long*>(&vtag[st][b]);
+    unsigned long long w = *tag;
+    if ((int)(uint32_t)w != t) {
+      const uint64_t t0 = globaltimer_ns();
+      uint64_t limit = 0;
+      for (uint32_t spins = 1; (int)(uint32_t)(w = *tag) != t; ++spins) {
+        if ((spins & 63u) == 0) {
+          if (*abort_flag) return false;
+          if (limit == 0) limit = wait_limit_ns(err);
+          if (globaltimer_ns() - t0 > limit || spins >= kWaitMaxPolls) {
+            record_error(err, kDevTimeoutMbarrier);
+            *abort_flag = 1;
+            return false;
+          }
+        }
+      }
+    }
+    e[b] = (int)(uint32_t)(w >> 32);
+  }
+  return true;
+}
+
+// SAFE = false: the fast instance.  V enters the PV products as it is (fp16
+// holds |v| in [2^-6, 2^15) with full precision); a unit whose V reaches
+// outside that range leaves a marker in its output and is recomputed by the
+// SAFE instance, launched right after on the same stream, which takes only the
+// marked units and carries V as block floating point (see the header comment).
+template <int D, typename OutT, bool VARLEN, bool SAFE>
 __global__ void __launch_bounds__(kThreads, 1)
     plx_prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                           const __grid_constant__ CUtensorMap rmap,
@@ -249,8 +319,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bars* bars = reinterpret_cast<Bars*>(xch + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* umask = reinterpret_cast<uint32_t*>(tmem_slot + 4);  // SAFE: kMaskUnits bits
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if constexpr (SAFE) {
+    // find this CTA's marked units; a CTA with none returns at once
+    for (int w = tid; w < kMaskUnits / 32; w += kThreads) umask[w] = 0u;
+    __syncthreads();
+    int any = 0;
+    for (int k = tid; k < kMaskUnits; k += kThreads) {
+      const long long u = blockIdx.x + (long long)k * gridDim.x;
+      if (u >= p.units) break;
+      const Unit x = unit_of<VARLEN>(p, (int)u);
+      if (x.n > 0 &&
+          is_marked<OutT>(p.out, (((size_t)x.tok0 + x.mt * kBM) * p.Hq + x.h) * D)) {
+        atomicOr(&umask[k >> 5], 1u << (k & 31));
+        any = 1;
+      }
+    }
+    if (!__syncthreads_or(any)) return;
+  }
 
   if (tid == 0) {
     *abort_flag = 0;
@@ -266,7 +355,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->s_free, kSoftWarps);  // one arrival per softmax warp
     mbar_init(&bars->p_full, kSoftWarps);
     mbar_init(&bars->o_done, 1);
-    mbar_init(&bars->conv_sync, kConvWarps);
+    mbar_init(&bars->v_reload[0], 1);
+    mbar_init(&bars->v_reload[1], 1);
+    mbar_init(&bars->v_rescaled, kSoftWarps);
+    for (int s = 0; s < kStages; ++s) bars->vtag[s][0] = bars->vtag[s][1] = make_int2(-1, 0);
+    for (int s = 0; s < 8; ++s) bars->vunit[s][0] = bars->vunit[s][1] = make_int2(-1, 0);
     fence_mbarrier_init();
   }
   {
@@ -297,11 +390,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ku counts the units with work (varlen units past a sequence's last
       // query tile have none); every role counts them the same way
       for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-        const Unit x = unit_of<VARLEN>(p, u);
+        const Unit x = unit_at<VARLEN, SAFE>(p, u, umask);
         if constexpr (VARLEN) {
-          if (x.bad && x.mt == 0) record_error(p.err, kDevBadArgument);
-          if (x.n == 0) continue;
+          if (!SAFE && x.bad && x.mt == 0) record_error(p.err, kDevBadArgument);
         }
+        if (x.n == 0) continue;
         const int hk = x.h / p.G;
         if (ku > 0 && !mbar_wait(&bars->q_empty, (ku - 1) & 1, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&bars->q_full, 2 * C::Q_BYTES);
@@ -313,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (u + (int)gridDim.x < p.units) {
           // the next unit's Q and R come from L2 when the Q/R buffers free up
-          const Unit y = unit_of<VARLEN>(p, u + gridDim.x);
+          const Unit y = unit_at<VARLEN, SAFE>(p, u + gridDim.x, umask);
           if (y.n > 0) {
             for (int kb = 0; kb < C::KB; ++kb) {
               tma_prefetch_l2_4d(&qmap, kb * 64, y.h, y.row0 + y.mt * kBM, y.bc);
@@ -360,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t = 0, ku = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-        const int n = unit_of<VARLEN>(p, u).n;
+        const int n = unit_at<VARLEN, SAFE>(p, u, umask).n;
         if (n == 0) continue;
         for (int j = 0; j < n; ++j, ++t) {
           const int st = t % kStages;
@@ -403,16 +496,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int st = 0; st < kStages; ++st)
         dv[st] = smem_desc_sw128(smem_u32(sKV + C::v_box(st, 0)), C::v_lbo(st), 1024);
-      int t = 0;
+      int t = 0, rescales = 0;
+      int pe[2] = {0, 0};  // block exponents of the previous tile's V
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-        const int n = unit_of<VARLEN>(p, u).n;
+        const int n = unit_at<VARLEN, SAFE>(p, u, umask).n;
         for (int j = 0; j < n; ++j, ++t) {
           const int st = t % kStages;
           if (!mbar_wait(&bars->p_full, t & 1, abort_flag, p.err) ||
               !mbar_wait(&bars->v_ready[st], (t / kStages) & 1, abort_flag, p.err)) {
             ok = false;
             break;
+          }
+          if constexpr (SAFE) {
+            // a tile whose V needed another block exponent than the previous
+            // one waits until the softmax warps have rescaled O and U
+            int e[2];
+            read_vtags<C::KB>(bars->vtag, t, e, abort_flag, p.err);  // posted before v_ready
+            if (j > 0 && (e[0] != pe[0] || e[1] != pe[1])) {
+              if (!mbar_wait(&bars->v_rescaled, rescales & 1, abort_flag, p.err)) {
+                ok = false;
+                break;
+              }
+              ++rescales;
+            }
+            pe[0] = e[0];
+            pe[1] = e[1];
           }
           tc_fence_after();
           uint64_t bv = dv[0];
@@ -441,92 +550,128 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2 || warp == kConvWarp2) {
     // ------------------------------------------------------------ V converters
     // V of each tile -> fp16 in place (the PV products run in fp16), scaled by
-    // 2^-E (block floating point, E the unit's running block exponent).  Each
-    // of the two converter warps takes half of the tile's 16-byte words: a
-    // first pass finds its half's largest |v| (bf16 magnitudes, packed max),
-    // the halves are combined through shared memory, a second pass scales (if
-    // E != 0) and converts, eight words per thread at a time.
-    constexpr int kWords = C::KV_BYTES / 16;         // 16-byte words of a V tile
-    constexpr int kIters = kWords / (2 * 32 * 8);    // per converter, 8 words per step
-    static_assert(kIters >= 1 && kWords % (2 * 32 * 8) == 0, "converter split");
-    const int cw = warp == 2 ? 0 : 1;                // which half of the words
-    int g = 0;
+    // 2^-E (block floating point).  Converter warp cw owns V column block cw
+    // (d = 64: one block, converter 1 only signals) and its own running block
+    // exponent E over the unit's tiles.  It converts the block with the current
+    // E, eight 16-byte words per thread at a time, while finding its largest
+    // |v|.  If the block asks for another E (the unit's first tile outside
+    // the range fp16 holds as it is, or a later tile that needs a larger E),
+    // the block is fetched again by TMA and converted with the new E: a rare
+    // path, taken only by data far outside fp16's range.  The E is posted with
+    // the tile number (vtag), then v_ready releases the tile to the PV products.
+    constexpr int kBlockWords = C::KV_BOX / 16;       // 16-byte words of one column block
+    constexpr int kIters = kBlockWords / (32 * 8);    // 8 words per thread per step
+    static_assert(kBlockWords % (32 * 8) == 0, "converter steps");
+    const int cw = warp == 2 ? 0 : 1;                 // the column block of this warp
+    const bool has_block = cw < C::KB;
+    int g = 0, reloads = 0, uc = 0;  // uc: units with work so far
     bool ok = true;
+    if (lane == 0) tma_prefetch_desc(&vmap);
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-      const int n = unit_of<VARLEN>(p, u).n;
-      int ve = kVExpMin;
+      const Unit x = unit_at<VARLEN, SAFE>(p, u, umask);
+      const int n = x.n;
+      const int hk = x.h / p.G;
+      int ve = 0;       // this block's running exponent in the unit (0: V as it is)
+      float umax = 0.f;  // fast instance: the unit's largest |v| in this block
       for (int j = 0; j < n; ++j) {
         const int t = g + j, st = t % kStages;
         if (!mbar_wait(&bars->kv_full[st], (t / kStages) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
-        // word w of the tile: column block w / 512, word w % 512 of it
-        auto word = [&](int h, int q) {
-          const int w = (cw * kIters + h) * 256 + 32 * q + lane;
-          return reinterpret_cast<uint4*>(sKV + C::v_box(st, w >> 9)) + (w & 511);
-        };
-        uint32_t mx = 0;
+        uint4* blk = reinterpret_cast<uint4*>(sKV + C::v_box(st, has_block ? cw : 0));
+        // converts the block with 2^-e; returns this thread's largest |v|
+        auto convert = [&](int e) {
+          const float sc = __int_as_float((127 - e) << 23);  // 2^-e, exact
+          const float2 sc2 = make_float2(sc, sc);
+          float mx = 0.f;
 #pragma unroll 1
-        for (int h = 0; h < kIters; ++h) {
+          for (int h = 0; h < kIters; ++h) {
+            uint4 w[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 w = *word(h, q);
-            mx = bf16x2_max(mx, bf16x2_max(bf16x2_max(w.x & 0x7fff7fffu, w.y & 0x7fff7fffu),
-                                           bf16x2_max(w.z & 0x7fff7fffu, w.w & 0x7fff7fffu)));
-          }
-        }
-        mx = __reduce_max_sync(0xffffffffu, max(mx & 0xffffu, mx >> 16));
-        // combine with the other converter's half (slots alternate by tile,
-        // so one arrival per tile and converter suffices)
-        if (lane == 0) {
-          xch->vmax[t & 1][cw] = mx;
-          mbar_arrive(&bars->conv_sync);
-        }
-        if (!mbar_wait(&bars->conv_sync, t & 1, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
-        mx = max(xch->vmax[t & 1][0], xch->vmax[t & 1][1]);
-        if (mx != 0) {
-          // floor(log2 |v|max) from the bf16 exponent field (subnormals count as
-          // 2^-127, inf and NaN as 2^128: those results are reported anyway)
-          const int fl = (int)(mx >> 7) - 127;
-          const int e = (fl >= kVLowBits && fl <= kVHeadroomBits)
-                            ? 0
-                            : min(kVExpMax, max(kVExpMin, fl - kVHeadroomBits));
-          ve = max(ve, e);
-        }
-        const int vuse = max(ve, kVExpMin);
-        const float sc = __int_as_float((127 - vuse) << 23);  // 2^-E, exact
-        const float2 sc2 = make_float2(sc, sc);
-        const bool scaled = vuse != 0;
-#pragma unroll 1
-        for (int h = 0; h < kIters; ++h) {
-          uint4 w[8];
+            for (int q = 0; q < 8; ++q) w[q] = blk[h * 256 + 32 * q + lane];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) w[q] = *word(h, q);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float2 f0 = bf16x2_to_float2(w[q].x), f1 = bf16x2_to_float2(w[q].y);
-            float2 f2v = bf16x2_to_float2(w[q].z), f3 = bf16x2_to_float2(w[q].w);
-            if (scaled) {
-              f0 = __fmul2_rn(f0, sc2);
-              f1 = __fmul2_rn(f1, sc2);
-              f2v = __fmul2_rn(f2v, sc2);
-              f3 = __fmul2_rn(f3, sc2);
+            for (int q = 0; q < 8; ++q) {
+              float2 f0 = bf16x2_to_float2(w[q].x), f1 = bf16x2_to_float2(w[q].y);
+              float2 f2v = bf16x2_to_float2(w[q].z), f3 = bf16x2_to_float2(w[q].w);
+              mx = fmax3(mx, fabsf(f0.x), fabsf(f0.y));
+              mx = fmax3(mx, fabsf(f1.x), fabsf(f1.y));
+              mx = fmax3(mx, fabsf(f2v.x), fabsf(f2v.y));
+              mx = fmax3(mx, fabsf(f3.x), fabsf(f3.y));
+              if (e != 0) {
+                f0 = __fmul2_rn(f0, sc2);
+                f1 = __fmul2_rn(f1, sc2);
+                f2v = __fmul2_rn(f2v, sc2);
+                f3 = __fmul2_rn(f3, sc2);
+              }
+              w[q] = make_uint4(float2_to_f16x2(f0.x, f0.y), float2_to_f16x2(f1.x, f1.y),
+                                float2_to_f16x2(f2v.x, f2v.y), float2_to_f16x2(f3.x, f3.y));
+              blk[h * 256 + 32 * q + lane] = w[q];
             }
-            w[q] = make_uint4(float2_to_f16x2(f0.x, f0.y), float2_to_f16x2(f1.x, f1.y),
-                              float2_to_f16x2(f2v.x, f2v.y), float2_to_f16x2(f3.x, f3.y));
-            *word(h, q) = w[q];
           }
+          return mx;
+        };
+        if (!SAFE) {
+          // fast instance: V as it is; the unit's largest |v| decides whether
+          // the unit is handed to the recomputing instance
+          if (has_block) {
+            const float mx =
+                __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(convert(0))));
+            umax = j == 0 ? mx : fmaxf(umax, mx);
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+          if (j == n - 1 && lane == 0) {
+            // out of range: nonzero and below 2^kVLowBits, at least
+            // 2^(kVHeadroomBits + 1), or not finite
+            const bool oor = has_block && umax > 0.f &&
+                             !(umax >= exp2f((float)kVLowBits) &&
+                               umax < exp2f((float)(kVHeadroomBits + 1)));
+            *reinterpret_cast<volatile unsigned long long*>(&bars->vunit[uc & 7][cw]) =
+                (unsigned long long)(uint32_t)uc | ((unsigned long long)(oor ? 1u : 0u) << 32);
+          }
+        } else if (has_block) {
+          const int used = j == 0 ? 0 : ve;
+          // warp max (|v| >= 0: its fp32 bits order like the values)
+          const float mx =
+              __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(convert(used))));
+          // the exponent this block asks for: 0 while its largest |v| lies in
+          // [2^kVLowBits, 2^(kVHeadroomBits + 1)); else floor(log2 max) - 14
+          // (inf and NaN count as 2^128: their results are reported anyway)
+          int e = 0;
+          if (mx > 0.f) {
+            const int fl = isfinite(mx) ? ((int)((__float_as_uint(mx) >> 23) & 0xff) - 127) : 128;
+            if (fl < kVLowBits || fl > kVHeadroomBits)
+              e = min(kVExpMax, max(kVExpMin, fl - kVHeadroomBits));
+          }
+          const int want = j == 0 ? e : max(ve, e);
+          if (want != used) {
+            // converted with the wrong scale: fetch the block again and redo
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&bars->v_reload[cw], C::KV_BOX);
+              tma_load_4d(sKV + C::v_box(st, cw), &vmap, &bars->v_reload[cw], cw * 64, hk,
+                          x.row0 + j * kBN, x.bc);
+            }
+            if (!mbar_wait(&bars->v_reload[cw], reloads & 1, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            ++reloads;
+            convert(want);
+          }
+          ve = want;
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0)  // one 8-byte write: (tile, E)
+            *reinterpret_cast<volatile unsigned long long*>(&bars->vtag[st][cw]) =
+                (unsigned long long)(uint32_t)t | ((unsigned long long)(uint32_t)ve << 32);
         }
-        if (cw == 0 && lane == 0) bars->vexp[st] = vuse;
-        fence_proxy_async_smem();
-        __syncwarp();
         if (lane == 0) mbar_arrive(&bars->v_ready[st]);
       }
       g += n;
+      if (n > 0) ++uc;
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -538,20 +683,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t my_cols = (uint32_t)(half * kHalf);  // first S/T column of this half
     const int bar_id = 1 + qd;                     // named barrier of the row's two warps
     const bool qpos = p.qscale >= 0.f;
-    int g = 0, xs = 0;
+    int g = 0, xs = 0, uc = 0;  // uc: units with work so far
     bool ok = true, finite = true;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-      const Unit x = unit_of<VARLEN>(p, u);
+      const Unit x = unit_at<VARLEN, SAFE>(p, u, umask);
       if (x.n == 0) continue;  // (varlen) no such query tile
       const int i = x.mt * kBM + r;
       // Running max m (log2 units of the scaled scores); P = 2^(s - m) <= 2^8
       // (lazy rescaling).  eu (>= 0) keeps P t 2^-eu in fp16's range.
       float m_run = -INFINITY;
       int eu = 0;
-      int ve = 0;  // block exponent of the V columns of O and U (see the converter)
+      // block exponents of the V column blocks of O and U (see the converters)
+      int ve[2] = {0, 0};
       float tlim = (float)(1 << kTBits), tsc = 1.f;  // 2^(kTBits + eu), 2^-eu
+      // Tile t-1's block exponents, checked one tile late (the converters are
+      // long done by then): where they changed, PV of t-1 waits until O and U
+      // (V columns only) have been brought to the new scale here.
+      auto v_check = [&](int tp, int jp) {
+        int e[2];
+        if (!read_vtags<C::KB>(bars->vtag, tp, e, abort_flag, p.err)) return false;
+        if (jp > 0 && (e[0] != ve[0] || e[1] != ve[1])) {
+          const uint32_t base = lane_addr + (half == 0 ? C::COL_O : C::COL_U);
+          const float f0 = exp2f((float)(ve[0] - e[0])), f1 = exp2f((float)(ve[1] - e[1]));
+#pragma unroll 1
+          for (int cc = 0; cc < D; cc += 64) {
+            const float f = cc < 64 ? f0 : f1;
+            uint32_t wa[32], wb[32];
+            tmem_ld2x32_sync(base + cc, base + cc + 32, wa, wb);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              wa[q] = __float_as_uint(__uint_as_float(wa[q]) * f);
+              wb[q] = __float_as_uint(__uint_as_float(wb[q]) * f);
+            }
+            tmem_st32(base + cc, wa);
+            tmem_st32(base + cc + 32, wb);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->v_rescaled);
+        }
+        ve[0] = e[0];
+        ve[1] = e[1];
+        return true;
+      };
       for (int j = 0; j < x.n; ++j) {
         const int t = g + j;
+        if (SAFE && j > 0 && !v_check(t - 1, j - 1)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait(&bars->s_full, t & 1, abort_flag, p.err)) {
           ok = false;
           break;
@@ -609,21 +790,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         int eu_new = eu;
         if (tmax >= tlim) eu_new = max(eu, (int)ceilf(log2f(tmax)) - (kTBits - 1));
         const bool ubump = eu_new > eu;
-        // the block exponent the converter scaled this tile's V by
-        const int st = t % kStages;
-        if (!mbar_wait(&bars->v_ready[st], (t / kStages) & 1, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
-        const int ve_new = bars->vexp[st];
-        const bool vchange = j > 0 && ve_new != ve;  // the same for every thread of the CTA
-        float vf = 1.f;  // factor of the V columns of O and U (not of l, z)
-        if (vchange) vf = exp2f((float)(ve - ve_new));
-        ve = ve_new;
         // O and U (with l, z) are rescaled below, after P and P t are stored;
         // P and P t already use the new m and eu.  (The partner warp holds the
         // same rows, so both warps of a row take the branch together.)
-        const bool rescale = __any_sync(0xffffffffu, resc || ubump) || vchange;
+        const bool rescale = __any_sync(0xffffffffu, resc || ubump);
         float fr = 1.f;  // this half's factor: half 0 rescales O (and l), half 1 U (and z)
         if (rescale) {
           const float alpha = resc ? exp2f(m_run - m_new) : 1.f;
@@ -685,15 +855,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st16(lane_addr + C::COL_PT + my_cols / 2, pk);
         if (rescale) {
           const uint32_t base = lane_addr + (half == 0 ? C::COL_O : C::COL_U);
-          const float frv = fr * vf;  // the V columns; the ones columns take fr
 #pragma unroll 1
           for (int cc = 0; cc < D; cc += 64) {
             uint32_t wa[32], wb[32];
             tmem_ld2x32_sync(base + cc, base + cc + 32, wa, wb);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              wa[e] = __float_as_uint(__uint_as_float(wa[e]) * frv);
-              wb[e] = __float_as_uint(__uint_as_float(wb[e]) * frv);
+              wa[e] = __float_as_uint(__uint_as_float(wa[e]) * fr);
+              wb[e] = __float_as_uint(__uint_as_float(wb[e]) * fr);
             }
             tmem_st32(base + cc, wa);
             tmem_st32(base + cc + 32, wb);
@@ -713,6 +882,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: out = ((1 + z/l) o - u) / l, lse = ln(sum exp(scale s));
       // l and z are the ones-columns of O and U; each half writes half the row.
       const int tl = g + x.n - 1;
+      if (SAFE && !v_check(tl, x.n - 1)) break;
+      bool oor = false;  // fast instance: this unit's V is out of range (marker)
+      if constexpr (!SAFE) {
+        // posted by the converters with the unit count once the unit's last V
+        // tile was converted (long ago by now)
+        for (int c = 0; c < C::KB; ++c) {
+          volatile const unsigned long long* tag =
+              reinterpret_cast<volatile const unsigned long long*>(&bars->vunit[uc & 7][c]);
+          unsigned long long w = *tag;
+          const uint64_t t0 = globaltimer_ns();
+          for (uint32_t spins = 1; (int)(uint32_t)w != uc; ++spins) {
+            if ((spins & 63u) == 0 &&
+                (*abort_flag || globaltimer_ns() - t0 > wait_limit_ns(p.err) ||
+                 spins >= kWaitMaxPolls)) {
+              if (!*abort_flag) record_error(p.err, kDevTimeoutMbarrier);
+              *abort_flag = 1;
+              break;
+            }
+            w = *tag;
+          }
+          if ((int)(uint32_t)w != uc) {
+            ok = false;
+            break;
+          }
+          oor = oor || (w >> 32) != 0;
+        }
+        if (!ok) break;
+        ++uc;
+      }
       if (!mbar_wait(&bars->o_done, tl & 1, abort_flag, p.err)) break;
       tc_fence_after();
       uint32_t lw, zw;
@@ -720,19 +918,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float l = __uint_as_float(lw), z = __uint_as_float(zw);
       const float inv = 1.f / l;
       const float usc = exp2f((float)eu);           // undo the P t scaling
-      const float vsc = exp2f((float)ve);           // and the block scaling of V
-      const float c1 = (1.f + z * usc * inv) * inv * vsc;
-      const float cu = usc * inv * vsc;
+      const float c1 = (1.f + z * usc * inv) * inv;
+      const float cu = usc * inv;
+      const float vsc0 = exp2f((float)ve[0]), vsc1 = exp2f((float)ve[1]);
       OutT* orow = static_cast<OutT*>(p.out) + (((size_t)x.tok0 + i) * p.Hq + x.h) * D;
 #pragma unroll 1
       for (int cc = half * (D / 2); cc < (half + 1) * (D / 2); cc += 32) {
         uint32_t ov[32], uv[32];
         tmem_ld2x32_sync(lane_addr + C::COL_O + cc, lane_addr + C::COL_U + cc, ov, uv);
+        const float vsc = cc < 64 ? vsc0 : vsc1;  // undo the block scaling of V
+        const float c1v = c1 * vsc, cuv = cu * vsc;
         float a[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          a[e] = __uint_as_float(ov[e]) * c1 - __uint_as_float(uv[e]) * cu;
-          finite = finite && isfinite(a[e]);
+          a[e] = __uint_as_float(ov[e]) * c1v - __uint_as_float(uv[e]) * cuv;
+          finite = finite && (oor || isfinite(a[e]));
         }
         if (i < x.len) {
           if constexpr (sizeof(OutT) == 2) {
@@ -753,6 +953,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (half == 0 && p.lse && i < x.len)
         p.lse[x.lse0 + i] = (m_run + log2f(l)) * 0.6931471805599453f;
+      if (oor && half == 0 && r == 0) {
+        // hand the unit to the recomputing instance (its first row, column 0;
+        // the row itself is rewritten there)
+        if constexpr (sizeof(OutT) == 2)
+          reinterpret_cast<uint16_t*>(orow)[0] = kMarkBf16;
+        else
+          reinterpret_cast<uint32_t*>(orow)[0] = kMarkF32;
+      }
       tc_fence_before();
       g += x.n;
     }
@@ -811,12 +1019,28 @@ cudaError_t launch_d(const PrefillTcArgs& a, cudaStream_t stream) {
   p.err = a.err;
   p.cu_seqlens = a.cu_seqlens;
   p.total = a.total;
-  const int smem = 1024 + C::TILE_SMEM + (int)sizeof(Xchg) + (int)sizeof(Bars) + 16;
-  auto kern = plx_prefill_tc_kernel<D, OutT, VARLEN>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem =
+      1024 + C::TILE_SMEM + (int)sizeof(Xchg) + (int)sizeof(Bars) + 16 + kMaskUnits / 8;
+  static_assert(1024 + TcCfg<D>::TILE_SMEM + sizeof(Xchg) + sizeof(Bars) + 16 + kMaskUnits / 8 <=
+                    227 * 1024,
+                "shared memory");
+  // the fast instance over every unit ...
+  auto fast = plx_prefill_tc_kernel<D, OutT, VARLEN, false>;
+  e = cudaFuncSetAttribute(fast, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = (int)(units < a.num_sms ? units : a.num_sms);
-  kern<<<grid, kThreads, smem, stream>>>(qm, rm, km, vm, p);
+  fast<<<grid, kThreads, smem, stream>>>(qm, rm, km, vm, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // ... then the recomputing instance over the units it marked (a CTA with no
+  // marked unit returns after one read per unit)
+  auto safe = plx_prefill_tc_kernel<D, OutT, VARLEN, true>;
+  e = cudaFuncSetAttribute(safe, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  long long sgrid = (units + kMaskUnits - 1) / kMaskUnits;
+  if (sgrid < grid) sgrid = grid;
+  if (sgrid > 0x7fffffffll) return cudaErrorInvalidValue;
+  safe<<<(unsigned)sgrid, kThreads, smem, stream>>>(qm, rm, km, vm, p);
   return cudaGetLastError();
 }
 
