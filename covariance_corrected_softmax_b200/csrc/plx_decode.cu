@@ -171,25 +171,62 @@ __device__ __forceinline__ uint32_t swz_off(int row, int c) {
   return (uint32_t)((c >> 3) * BOX_BYTES + row * 128 + (((c & 7) ^ (row & 7)) << 4));
 }
 
+// The result of row (b, h), element c, from its merged softmax sums:
+// out = (1 + tbar) o - u with tbar = Z/L, o = O/L, u = U/L, or, in state mode,
+// the state (m, l, z, 0, o[D], u[D]) itself.
+template <typename T, int D, int MODE>
+__device__ __forceinline__ void write_result(const DecodeParams& p, int b, int h, int c, float M,
+                                             float L, float Z, float O, float U);
+
 // Kernel instances (see the main kernel).
 constexpr int kDecContiguous = 0, kDecPaged = 1, kDecState = 2;
 constexpr int kDecStateMode = kDecState;
 
+template <typename T, int D, int MODE>
+__device__ __forceinline__ void write_result(const DecodeParams& p, int b, int h, int c, float M,
+                                             float L, float Z, float O, float U) {
+  constexpr int PHF = part_head_floats<D>();
+  if constexpr (MODE == kDecStateMode) {
+    float* sr = p.state + ((size_t)b * p.Hq + h) * PHF;
+    if (c == 0) {
+      sr[0] = M;
+      sr[1] = L;
+      sr[2] = Z;
+      sr[3] = 0.f;
+    }
+    sr[4 + c] = O;
+    sr[4 + D + c] = U;
+  } else {
+    const float inv = 1.f / L;
+    const float val = ((1.f + Z * inv) * O - U) * inv;
+    store_elem<T>(p.out, ((size_t)b * p.Hq + h) * D + c, val);
+  }
+}
+
 // ---------------------------------------------------------------------------
-// Segment finalisation: merge the NW consumer warps' states of a head group
-// (in shared memory: [warp][head] m, l, z, pad, o[D], u[D]) with the
-// log-sum-exp rule, then write the output (a segment complete in this CTA),
-// the row's softmax state (state mode), or this CTA's partial slot with its
-// header (a segment split across CTAs; the combine kernel merges the pieces).
+// Segment finalisation.  The NW consumer warps' states of a head group (in
+// shared memory: [warp][head] m, l, z, pad, o[D], u[D]) are merged with the
+// log-sum-exp rule; then
+//  * a segment whose tiles all ran in this CTA writes its output (or, in state
+//    mode, the row's softmax state);
+//  * a piece of a segment split across CTAs goes to one of this CTA's two
+//    workspace slots (slot 0: the CTA's first segment, slot 1: its last); a
+//    piece that does not end the segment is published with a header
+//    (segment, call tag) written after the data;
+//  * the piece that ends a split segment (necessarily the CTA's first
+//    segment) is merged with the earlier pieces once the CTA has finished all
+//    its tiles (merge_tail below): every CTA holds about the same work, so the
+//    CTAs holding those pieces finish at about the same time.
 // Called by all consumer threads between two consumer-wide barriers.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int HPW, int MODE, int NW>
 __device__ __forceinline__ void finalize_segment(const DecodeParams& p, const TileMeta& mt, int h0,
-                                                 bool complete, float* part,
-                                                 const float* merge, int tid) {
+                                                 float* part, const float* merge, int tid) {
   constexpr int PHF = part_head_floats<D>();
-  for (int pr = tid; pr < HPW * D; pr += NW * 32) {
-    const int g = pr / D, c = pr % D;
+  static_assert(HPW * D <= NW * 32, "one element per consumer thread");
+  const bool starts = (mt.flags & 4) != 0, ends = (mt.flags & 8) != 0;
+  const int g = tid / D, c = tid % D;  // one (head, column) per thread
+  if (tid < HPW * D) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) M = fmaxf(M, merge[(w * HPW + g) * PHF]);
@@ -203,21 +240,8 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams& p, const Ti
       O += wt * src[4 + c];
       U += wt * src[4 + D + c];
     }
-    if (MODE == kDecStateMode && complete) {
-      float* sr = p.state + ((size_t)mt.b * p.Hq + h0 + g) * PHF;
-      if (c == 0) {
-        sr[0] = M;
-        sr[1] = L;
-        sr[2] = Z;
-        sr[3] = 0.f;
-      }
-      sr[4 + c] = O;
-      sr[4 + D + c] = U;
-    } else if (complete) {
-      // out = (1 + tbar) o - u with tbar = Z/L, o = O/L, u = U/L
-      const float inv = 1.f / L;
-      const float val = ((1.f + Z * inv) * O - U) * inv;
-      store_elem<T>(p.out, ((size_t)mt.b * p.Hq + h0 + g) * D + c, val);
+    if (starts && ends) {
+      write_result<T, D, MODE>(p, mt.b, h0 + g, c, M, L, Z, O, U);
     } else {
       float* ph = part + kPartHeader + g * PHF;
       if (c == 0) {
@@ -229,13 +253,87 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams& p, const Ti
       ph[4 + D + c] = U;
     }
   }
-  if (!complete && tid == 0) {
-    int* hdr = reinterpret_cast<int*>(part);
-    hdr[1] = (mt.flags & 4) ? 1 : 0;
-    hdr[2] = (mt.flags & 8) ? 1 : 0;
-    hdr[3] = 0;
-    hdr[0] = mt.seg;
+  if (!ends) {
+    // publish: the data above, then the header
+    __threadfence();
+    named_bar_sync(1, NW * 32);
+    if (tid == 0) {
+      volatile int* hdr = reinterpret_cast<volatile int*>(part);
+      hdr[1] = starts ? 1 : 0;
+      hdr[2] = 0;
+      hdr[3] = p.call_tag;
+      __threadfence();
+      hdr[0] = mt.seg;
+    }
   }
+}
+
+// The split segment whose last piece this CTA holds (in its slot 0): merge the
+// pieces CTA by CTA from the one where the segment began (each found by its
+// header, waited for with a bounded spin: all CTAs of the grid are resident,
+// one per SM, and a piece never waits for a later one), this CTA's last, and
+// write the output or state.  Called by all consumer threads after the tiles.
+template <typename T, int D, int HPW, int MODE, int NW>
+__device__ __forceinline__ void merge_tail(const DecodeParams& p, int b, int seg, int h0,
+                                           long long seg_t0, long long total, int tid,
+                                           volatile int* abort_flag, int* found_slot) {
+  constexpr int PF = part_floats<D>(HPW);
+  constexpr int PHF = part_head_floats<D>();
+  const float* base = p.ws + kWsHeaderFloats;
+  long long cf = seg_t0 * p.grid / total;
+  while (cf > 0 && total * cf / p.grid > seg_t0) --cf;
+  while (cf + 1 < p.grid && total * (cf + 1) / p.grid <= seg_t0) ++cf;
+  const int g = tid / D, c = tid % D;
+  const bool act = tid < HPW * D;
+  float M = -INFINITY, L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
+  auto absorb = [&](const float* ph) {
+    const float m = __ldcg(ph);
+    const float Mn = fmaxf(M, m);
+    const float wa = merge_weight(M, Mn), wb = merge_weight(m, Mn);
+    L = L * wa + __ldcg(ph + 1) * wb;
+    Z = Z * wa + __ldcg(ph + 2) * wb;
+    O = O * wa + __ldcg(ph + 4 + c) * wb;
+    U = U * wa + __ldcg(ph + 4 + D + c) * wb;
+    M = Mn;
+  };
+  for (int cta = (int)cf; cta <= (int)blockIdx.x; ++cta) {
+    // a CTA whose tile range is empty holds no piece
+    if (total * cta / p.grid == total * (cta + 1) / p.grid) continue;
+    int slot = 0;  // this CTA's own piece: slot 0
+    if (cta < (int)blockIdx.x) {
+      if (tid == 0) {
+        // the piece is in slot 1 of the CTA where the segment began when that
+        // CTA finished an earlier segment first, otherwise in slot 0
+        int sl = -1;
+        const uint64_t t0 = globaltimer_ns();
+        uint64_t limit = 0;
+        for (uint32_t spins = 0; sl < 0; ++spins) {
+          for (int s = 0; s < 2 && sl < 0; ++s) {
+            const volatile int* hdr =
+                reinterpret_cast<const volatile int*>(base + (size_t)(2 * cta + s) * PF);
+            if (hdr[0] == seg && hdr[3] == p.call_tag) sl = s;
+          }
+          if (sl < 0 && (spins & 63u) == 63u) {
+            if (*abort_flag) break;
+            if (limit == 0) limit = wait_limit_ns(p.err);
+            if (globaltimer_ns() - t0 > limit || spins >= kWaitMaxPolls) {
+              record_error(p.err, kDevTimeoutMbarrier);
+              *abort_flag = 1;
+              break;
+            }
+          }
+        }
+        __threadfence();  // the piece's data, published before its header, is read below
+        *found_slot = sl;
+      }
+      named_bar_sync(1, NW * 32);
+      slot = *found_slot;
+      named_bar_sync(1, NW * 32);
+      if (slot < 0) return;  // gave up (error recorded)
+    }
+    if (act) absorb(base + (size_t)(2 * cta + slot) * PF + kPartHeader + g * PHF);
+  }
+  if (act) write_result<T, D, MODE>(p, b, h0 + g, c, M, L, Z, O, U);
 }
 
 // ---------------------------------------------------------------------------
@@ -272,6 +370,7 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
   RangeInfo* info = reinterpret_cast<RangeInfo*>(empty + STAGES);
   long long* scan_ws = reinterpret_cast<long long*>(info + 1);   // 16 entries
   volatile int* abort_flag = reinterpret_cast<volatile int*>(scan_ws + 16);
+  int* found_slot = reinterpret_cast<int*>(scan_ws + 18);
   float* merge = reinterpret_cast<float*>(scan_ws + 20);
   float* red_smem = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(merge + NW * HPW * PHF) + 15) & ~uintptr_t(15));
@@ -281,11 +380,6 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
 
   if (tid == 0) {
     *abort_flag = 0;
-    // Invalidate this CTA's two partial slots; finalisation rewrites them.
-    int* s0 = reinterpret_cast<int*>(p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x) * PF);
-    int* s1 = reinterpret_cast<int*>(p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + 1) * PF);
-    s0[0] = -1;
-    s1[0] = -1;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NW);
@@ -293,9 +387,6 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     fence_mbarrier_init();
   }
   locate_range(p, TK, info, scan_ws);  // contains __syncthreads
-  // The combine kernel may be scheduled now; it waits for this grid to finish.
-  grid_dep_launch_dependents();
-  if (blockIdx.x == 0 && tid == 0) reinterpret_cast<long long*>(p.ws)[0] = info->total;
 
   // Batches with an empty context produce zeros (out = 0 for an empty key set),
   // or the empty state (m = -inf, everything else 0).
@@ -444,7 +535,11 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     uint32_t qa[KS][4];
     float acc[KS][4];
     float m_run = -INFINITY, lsum = 0.f, zsum = 0.f;
-    int ordinal = 0;  // segments finalised so far by this CTA
+    int ordinal = 0;        // segments finalised so far by this CTA
+    long long seg_t0 = 0;   // first tile (global order) of the current segment
+    int tail_seg = -1, tail_b = 0, tail_h0 = 0;  // the split segment ending here
+    long long tail_t0 = 0;
+    bool done = true;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
@@ -455,11 +550,15 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
 
     for (long long t = t0, i = 0; t < t1; ++t, ++i) {
       const int stage = (int)(i % STAGES);
-      if (!mbar_wait(&full[stage], (uint32_t)((i / STAGES) & 1), abort_flag, p.err)) break;
+      if (!mbar_wait(&full[stage], (uint32_t)((i / STAGES) & 1), abort_flag, p.err)) {
+        done = false;
+        break;
+      }
       const TileMeta mt = metas[stage];
       const int h0 = mt.hkv * p.G + mt.hg * HPW;  // first query head of the group
 
       if (mt.flags & 1) {  // first tile of a segment in this CTA: load q, rho; reset
+        seg_t0 = t - mt.kt;  // the segment's first tile in the global order
         const size_t row = ((size_t)mt.b * p.Hq + h0 + hh) * (D / 2);
         const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q) + row;
         const uint32_t* r32 = reinterpret_cast<const uint32_t*>(p.rho) + row;
@@ -604,15 +703,23 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
       }
       if (mt.flags & 2) {
         named_bar_sync(1, NW * 32);
-        const bool complete = (mt.flags & 4) && (mt.flags & 8);
         // slot 0 holds the CTA's first segment, which may have begun in an
         // earlier CTA; slot 1 its last, which may end in a later one
         float* part = p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + (ordinal == 0 ? 0 : 1)) * PF;
-        finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, complete, part, merge, tid);
+        finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, part, merge, tid);
         named_bar_sync(1, NW * 32);
+        if ((mt.flags & 8) && !(mt.flags & 4)) {  // this CTA holds a split segment's end
+          tail_seg = mt.seg;
+          tail_b = mt.b;
+          tail_h0 = h0;
+          tail_t0 = seg_t0;
+        }
         ++ordinal;
       }
     }
+    if (done && tail_seg >= 0)
+      merge_tail<T, D, HPW, MODE, NW>(p, tail_b, tail_seg, tail_h0, tail_t0, info->total, tid,
+                                      abort_flag, found_slot);
   } else {
     // ------------------------------------------------------------ consumers (fp32)
     const int hw = lane >> 4, sub = lane & 15;
@@ -633,7 +740,11 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     float2 qf[HPW][H2], rf[HPW][H2], oa[HPW][H2], ua[HPW][H2];
     // running max of this lane's head, and l (score lanes) or z (probe lanes)
     float m_run = -INFINITY, lz = 0.f;
-    int ordinal = 0;  // segments finalised so far by this CTA
+    int ordinal = 0;        // segments finalised so far by this CTA
+    long long seg_t0 = 0;   // first tile (global order) of the current segment
+    int tail_seg = -1, tail_b = 0, tail_h0 = 0;  // the split segment ending here
+    long long tail_t0 = 0;
+    bool done = true;
 #pragma unroll
     for (int g = 0; g < HPW; ++g) {
 #pragma unroll
@@ -644,11 +755,15 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
 
     for (long long t = t0, i = 0; t < t1; ++t, ++i) {
       const int stage = (int)(i % STAGES);
-      if (!mbar_wait(&full[stage], (uint32_t)((i / STAGES) & 1), abort_flag, p.err)) break;
+      if (!mbar_wait(&full[stage], (uint32_t)((i / STAGES) & 1), abort_flag, p.err)) {
+        done = false;
+        break;
+      }
       const TileMeta mt = metas[stage];
       const int h0 = mt.hkv * p.G + mt.hg * HPW;  // first query head of the group
 
       if (mt.flags & 1) {  // first tile of a segment in this CTA: load q, rho; reset
+        seg_t0 = t - mt.kt;  // the segment's first tile in the global order
 #pragma unroll
         for (int g = 0; g < HPW; ++g) {
           const size_t base = ((size_t)mt.b * p.Hq + h0 + g) * D + sub * EPL;
@@ -823,95 +938,21 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
           }
         }
         named_bar_sync(1, NW * 32);
-        const bool complete = (mt.flags & 4) && (mt.flags & 8);
         float* part = p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + (ordinal == 0 ? 0 : 1)) * PF;
-        finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, complete, part, merge, tid);
+        finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, part, merge, tid);
         named_bar_sync(1, NW * 32);
+        if ((mt.flags & 8) && !(mt.flags & 4)) {  // this CTA holds a split segment's end
+          tail_seg = mt.seg;
+          tail_b = mt.b;
+          tail_h0 = h0;
+          tail_t0 = seg_t0;
+        }
         ++ordinal;
       }
     }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Combine kernel: one block per main-kernel CTA.  A block whose CTA holds the
-// head piece of a split segment merges that segment's pieces (the head piece,
-// then the first slot of each following CTA until the piece that ends it).
-// ---------------------------------------------------------------------------
-template <typename T, int D, int HPW>
-__global__ void __launch_bounds__(256)
-    plx_decode_combine_kernel(const DecodeParams p) {
-  constexpr int PF = part_floats<D>(HPW);
-  constexpr int PHF = part_head_floats<D>();
-  // launched as a programmatic dependent of the main kernel: wait for it
-  grid_dep_wait();
-  const float* base = p.ws + kWsHeaderFloats;
-  const int c0 = blockIdx.x;
-  int slot = -1;
-  for (int s = 1; s >= 0; --s) {
-    const int* hdr = reinterpret_cast<const int*>(base + (size_t)(2 * c0 + s) * PF);
-    if (hdr[0] >= 0 && hdr[1] == 1) {
-      slot = s;
-      break;
-    }
-  }
-  if (slot < 0) return;
-  const int* hdr0 = reinterpret_cast<const int*>(base + (size_t)(2 * c0 + slot) * PF);
-  const int seg = hdr0[0];
-  const int segs_per_b = p.Hkv * p.nhg;
-  const int b = seg / segs_per_b, seg_local = seg % segs_per_b;
-  const int hkv = seg_local / p.nhg, hg = seg_local % p.nhg;
-  const int h0 = hkv * p.G + hg * HPW;
-
-  for (int pr = threadIdx.x; pr < HPW * D; pr += blockDim.x) {
-    const int g = pr / D, c = pr % D;
-    float M = -INFINITY, L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
-    int cta = c0, s = slot;
-    bool ok = false;
-    while (cta < p.grid) {
-      const float* piece = base + (size_t)(2 * cta + s) * PF;
-      const int* hdr = reinterpret_cast<const int*>(piece);
-      if (hdr[0] == seg) {
-        const float* ph = piece + kPartHeader + g * PHF;
-        const float m = ph[0];
-        const float Mn = fmaxf(M, m);
-        const float wa = merge_weight(M, Mn), wb = merge_weight(m, Mn);
-        L = L * wa + ph[1] * wb;
-        Z = Z * wa + ph[2] * wb;
-        O = O * wa + ph[4 + c] * wb;
-        U = U * wa + ph[4 + D + c] * wb;
-        M = Mn;
-        if (hdr[2] == 1) {
-          ok = true;
-          break;
-        }
-      } else if (hdr[0] != -1 || cta == c0) {
-        // Tiles are contiguous: between two pieces of a segment there can only
-        // be CTAs that received no tiles at all (both slots invalid).
-        break;
-      }
-      ++cta;
-      s = 0;
-    }
-    if (!ok) {
-      record_error(p.err, kDevBadArgument);
-      continue;
-    }
-    if (p.state) {
-      float* sr = p.state + ((size_t)b * p.Hq + h0 + g) * PHF;
-      if (c == 0) {
-        sr[0] = M;
-        sr[1] = L;
-        sr[2] = Z;
-        sr[3] = 0.f;
-      }
-      sr[4 + c] = O;
-      sr[4 + D + c] = U;
-      continue;
-    }
-    const float inv = 1.f / L;
-    const float val = ((1.f + Z * inv) * O - U) * inv;
-    store_elem<T>(p.out, ((size_t)b * p.Hq + h0 + g) * D + c, val);
+    if (done && tail_seg >= 0)
+      merge_tail<T, D, HPW, MODE, NW>(p, tail_b, tail_seg, tail_h0, tail_t0, info->total, tid,
+                                      abort_flag, found_slot);
   }
 }
 
@@ -989,22 +1030,6 @@ cudaError_t launch_decode_t(const DecodeMaps& m, const DecodeParams& p, cudaStre
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<p.grid, Cfg::THREADS, smem, stream>>>(m.k, m.v, m.k_chunk, m.v_chunk, p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // The combine kernel is a programmatic dependent of the main kernel, so its
-  // launch overlaps the main kernel's tail (it waits for the main grid itself).
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.grid);
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, plx_decode_combine_kernel<T, D, HPW>, p);
-  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

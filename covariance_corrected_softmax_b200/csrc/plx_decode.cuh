@@ -16,7 +16,7 @@
 //    segments.  A persistent grid of CTAs splits the tile sequence into equal
 //    contiguous ranges (split-K with perfect balance for any mix of lengths);
 //    a segment that crosses a range boundary leaves partial states that the
-//    combine kernel merges with the log-sum-exp rule.
+//    CTA holding its last piece merges with the log-sum-exp rule.
 //  * One producer warp streams K and V tiles (TK keys x d) of the cache into a
 //    multi-stage shared-memory ring with TMA; the cache is read exactly once.
 //    A segment's last, partial tile is fetched in 16-row chunks, so rows past
@@ -90,7 +90,7 @@ template <int D>
 __host__ __device__ constexpr int part_floats(int hpw) {
   return kPartHeader + hpw * part_head_floats<D>();
 }
-constexpr int kWsHeaderFloats = 16;  // [0] = total tiles (int), rest reserved
+constexpr int kWsHeaderFloats = 16;  // reserved
 
 struct DecodeParams {
   const void* q;         // [B, Hq, D]
@@ -112,6 +112,10 @@ struct DecodeParams {
   // state over this cache -- m (log2 units of the scaled scores), l, z, 0,
   // o[D], u[D], unnormalised -- is written to state[(b * Hq + h) * (2D + 4)].
   float* state;
+  // Tag of this call (a host-side counter): a split segment's published
+  // pieces carry it, so a piece left in the workspace by an earlier call is
+  // never mistaken for this call's.
+  int call_tag;
 };
 
 // Tile metadata written by the producer next to each stage.

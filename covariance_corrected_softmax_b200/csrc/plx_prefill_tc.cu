@@ -324,6 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if constexpr (SAFE) {
+    // launched as a programmatic dependent of the fast instance: its output
+    // (with the markers) is visible once that grid has completed
+    grid_dep_wait();
     // find this CTA's marked units; a CTA with none returns at once
     for (int w = tid; w < kMaskUnits / 32; w += kThreads) umask[w] = 0u;
     __syncthreads();
@@ -377,6 +380,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  // the recomputing instance may be scheduled as SMs free up; it waits for
+  // this grid to complete before it reads anything this grid writes
+  if constexpr (!SAFE) grid_dep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -396,24 +402,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (x.n == 0) continue;
         const int hk = x.h / p.G;
-        if (ku > 0 && !mbar_wait(&bars->q_empty, (ku - 1) & 1, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(&bars->q_full, 2 * C::Q_BYTES);
-        for (int kb = 0; kb < C::KB; ++kb) {
-          tma_load_4d(sQ + kb * C::Q_BOX, &qmap, &bars->q_full, kb * 64, x.h,
-                      x.row0 + x.mt * kBM, x.bc);
-          tma_load_4d(sR + kb * C::Q_BOX, &rmap, &bars->q_full, kb * 64, x.h,
-                      x.row0 + x.mt * kBM, x.bc);
-        }
-        if (u + (int)gridDim.x < p.units) {
-          // the next unit's Q and R come from L2 when the Q/R buffers free up
-          const Unit y = unit_at<VARLEN, SAFE>(p, u + gridDim.x, umask);
-          if (y.n > 0) {
-            for (int kb = 0; kb < C::KB; ++kb) {
-              tma_prefetch_l2_4d(&qmap, kb * 64, y.h, y.row0 + y.mt * kBM, y.bc);
-              tma_prefetch_l2_4d(&rmap, kb * 64, y.h, y.row0 + y.mt * kBM, y.bc);
-            }
-          }
-        }
         for (int j = 0; j < x.n; ++j) {
           const int t = g + j, st = t % kStages;
           if (t >= kStages &&
@@ -427,6 +415,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                         x.row0 + j * kBN, x.bc);
             tma_load_4d(sKV + C::v_box(st, kb), &vmap, &bars->kv_full[st], kb * 64, hk,
                         x.row0 + j * kBN, x.bc);
+          }
+          if (j > 0) continue;
+          // Q and R of the unit, once its first K/V tile is on its way (that
+          // stage frees before the previous unit's last S/T products complete,
+          // which is what frees the Q/R buffers)
+          if (ku > 0 && !mbar_wait(&bars->q_empty, (ku - 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->q_full, 2 * C::Q_BYTES);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            tma_load_4d(sQ + kb * C::Q_BOX, &qmap, &bars->q_full, kb * 64, x.h,
+                        x.row0 + x.mt * kBM, x.bc);
+            tma_load_4d(sR + kb * C::Q_BOX, &rmap, &bars->q_full, kb * 64, x.h,
+                        x.row0 + x.mt * kBM, x.bc);
+          }
+          if (u + (int)gridDim.x < p.units) {
+            // the next unit's Q and R come from L2 when the Q/R buffers free up
+            const Unit y = unit_at<VARLEN, SAFE>(p, u + gridDim.x, umask);
+            if (y.n > 0) {
+              for (int kb = 0; kb < C::KB; ++kb) {
+                tma_prefetch_l2_4d(&qmap, kb * 64, y.h, y.row0 + y.mt * kBM, y.bc);
+                tma_prefetch_l2_4d(&rmap, kb * 64, y.h, y.row0 + y.mt * kBM, y.bc);
+              }
+            }
           }
         }
         g += x.n;
@@ -1040,7 +1053,18 @@ cudaError_t launch_d(const PrefillTcArgs& a, cudaStream_t stream) {
   long long sgrid = (units + kMaskUnits - 1) / kMaskUnits;
   if (sgrid < grid) sgrid = grid;
   if (sgrid > 0x7fffffffll) return cudaErrorInvalidValue;
-  safe<<<(unsigned)sgrid, kThreads, smem, stream>>>(qm, rm, km, vm, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)sgrid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, safe, qm, rm, km, vm, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

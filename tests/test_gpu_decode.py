@@ -159,6 +159,29 @@ def test_decode_rho_zero_is_softmax():
     check_out(to_np(out), ref, bf16=False, what="rho=0")
 
 
+@pytest.mark.parametrize("lens", [[200, 1, 300], [97, 1000, 5, 16], [4096, 1, 1, 1]],
+                         ids=["short", "mixed", "one_long"])
+def test_decode_lengths_far_below_capacity(lens):
+    """Lengths far below S_max: fewer key tiles than CTAs, so segments split
+    over CTAs with empty tile ranges between their pieces; the pieces must still
+    merge into the oracle's result (fp32 through the state path, and bf16)."""
+    B, Hq, Hkv, d, S = len(lens), 16, 8, 128, 4096
+    g = torch.Generator(device=DEV).manual_seed(sum(lens))
+    s = d ** -0.25
+    q = (torch.randn(B, Hq, d, generator=g, device=DEV) * s).to(torch.bfloat16)
+    rho = (torch.randn(B, Hq, d, generator=g, device=DEV) * 0.3).to(torch.bfloat16)
+    k = (torch.randn(B, S, Hkv, d, generator=g, device=DEV) * s).to(torch.bfloat16)
+    v = (torch.randn(B, S, Hkv, d, generator=g, device=DEV) * s).to(torch.bfloat16)
+    sl = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    out = plx.decode(q, rho, k, v, sl, softmax_scale=1.0)
+    st = plx.decode_state(q, rho, k, v, sl, softmax_scale=1.0)
+    f32 = plx.merge_states(st[None].contiguous(), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref, _ = oracle.decode(q, rho, k, v, sl, 1.0)
+    check_out(to_np(f32), ref, bf16=True, what=f"lengths {lens} (fp32 result)")
+    assert torch.equal(out, f32.to(torch.bfloat16))
+
+
 def test_decode_deterministic():
     shape = W.DecodeShape(B=8, Hq=16, Hkv=8, d=128, S_max=3000, ctx=3000, ragged=True)
     inp = W.make_decode(shape, seed=4, device=DEV)
