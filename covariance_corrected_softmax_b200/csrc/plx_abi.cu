@@ -4,7 +4,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cstddef>
 #include <mutex>
 
@@ -26,7 +25,6 @@ plx::EncodeTiledFn g_encode = nullptr;
 int g_sm_count[kMaxDevices] = {0};
 unsigned* g_err_ptr[kMaxDevices] = {nullptr};
 std::mutex g_dev_mu;
-std::atomic<unsigned> g_call_tag{1};  // decode call tags (see DecodeParams::call_tag)
 
 plx_status cuda_fail(cudaError_t e) {
   t_last_cuda_error = static_cast<int>(e);
@@ -290,7 +288,6 @@ plx_status decode_impl(const void* q, const void* rho, const void* k_new, const 
   p.page_size = pg.page_size;
   p.max_pages = pg.max_pages;
   p.state = state;
-  p.call_tag = (int)(g_call_tag.fetch_add(1u, std::memory_order_relaxed) & 0x7fffffffu);
   e = plx::launch_decode(bf16, d, maps, p, hpw, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return PLX_OK;

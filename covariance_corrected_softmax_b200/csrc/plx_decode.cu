@@ -212,7 +212,7 @@ __device__ __forceinline__ void write_result(const DecodeParams& p, int b, int h
 //  * a piece of a segment split across CTAs goes to one of this CTA's two
 //    workspace slots (slot 0: the CTA's first segment, slot 1: its last); a
 //    piece that does not end the segment is published with a header
-//    (segment, call tag) written after the data;
+//    (segment, launch tag) written after the data;
 //  * the piece that ends a split segment (necessarily the CTA's first
 //    segment) is merged with the earlier pieces once the CTA has finished all
 //    its tiles (merge_tail below): every CTA holds about the same work, so the
@@ -261,7 +261,7 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams& p, const Ti
       volatile int* hdr = reinterpret_cast<volatile int*>(part);
       hdr[1] = starts ? 1 : 0;
       hdr[2] = 0;
-      hdr[3] = p.call_tag;
+      hdr[3] = launch_tag();
       __threadfence();
       hdr[0] = mt.seg;
     }
@@ -269,71 +269,92 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams& p, const Ti
 }
 
 // The split segment whose last piece this CTA holds (in its slot 0): merge the
-// pieces CTA by CTA from the one where the segment began (each found by its
-// header, waited for with a bounded spin: all CTAs of the grid are resident,
-// one per SM, and a piece never waits for a later one), this CTA's last, and
-// write the output or state.  Called by all consumer threads after the tiles.
+// pieces of the CTAs from the one where the segment began, in CTA order, this
+// CTA's last, and write the output or state.  The earlier pieces are found by
+// their headers, one consumer thread per CTA waiting (bounded) for its piece:
+// all CTAs of the grid are resident, one per SM, and a piece never waits for a
+// later one.  Called by all consumer threads after the tiles; `slots` is
+// shared scratch of at least gridDim.x ints.
 template <typename T, int D, int HPW, int MODE, int NW>
 __device__ __forceinline__ void merge_tail(const DecodeParams& p, int b, int seg, int h0,
                                            long long seg_t0, long long total, int tid,
-                                           volatile int* abort_flag, int* found_slot) {
+                                           volatile int* abort_flag, int* slots) {
   constexpr int PF = part_floats<D>(HPW);
   constexpr int PHF = part_head_floats<D>();
   const float* base = p.ws + kWsHeaderFloats;
+  const int tag = launch_tag();
   long long cf = seg_t0 * p.grid / total;
   while (cf > 0 && total * cf / p.grid > seg_t0) --cf;
   while (cf + 1 < p.grid && total * (cf + 1) / p.grid <= seg_t0) ++cf;
-  const int g = tid / D, c = tid % D;
-  const bool act = tid < HPW * D;
-  float M = -INFINITY, L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
-  auto absorb = [&](const float* ph) {
-    const float m = __ldcg(ph);
-    const float Mn = fmaxf(M, m);
-    const float wa = merge_weight(M, Mn), wb = merge_weight(m, Mn);
-    L = L * wa + __ldcg(ph + 1) * wb;
-    Z = Z * wa + __ldcg(ph + 2) * wb;
-    O = O * wa + __ldcg(ph + 4 + c) * wb;
-    U = U * wa + __ldcg(ph + 4 + D + c) * wb;
-    M = Mn;
-  };
-  for (int cta = (int)cf; cta <= (int)blockIdx.x; ++cta) {
-    // a CTA whose tile range is empty holds no piece
-    if (total * cta / p.grid == total * (cta + 1) / p.grid) continue;
-    int slot = 0;  // this CTA's own piece: slot 0
-    if (cta < (int)blockIdx.x) {
-      if (tid == 0) {
-        // the piece is in slot 1 of the CTA where the segment began when that
-        // CTA finished an earlier segment first, otherwise in slot 0
-        int sl = -1;
-        const uint64_t t0 = globaltimer_ns();
-        uint64_t limit = 0;
-        for (uint32_t spins = 0; sl < 0; ++spins) {
-          for (int s = 0; s < 2 && sl < 0; ++s) {
-            const volatile int* hdr =
-                reinterpret_cast<const volatile int*>(base + (size_t)(2 * cta + s) * PF);
-            if (hdr[0] == seg && hdr[3] == p.call_tag) sl = s;
-          }
-          if (sl < 0 && (spins & 63u) == 63u) {
-            if (*abort_flag) break;
-            if (limit == 0) limit = wait_limit_ns(p.err);
-            if (globaltimer_ns() - t0 > limit || spins >= kWaitMaxPolls) {
-              record_error(p.err, kDevTimeoutMbarrier);
-              *abort_flag = 1;
-              break;
-            }
+  const int npieces = (int)blockIdx.x - (int)cf;  // earlier CTAs
+  for (int k = tid; k < npieces; k += NW * 32) {
+    const int cta = (int)cf + k;
+    int sl = -2;  // a CTA whose tile range is empty holds no piece
+    if (total * cta / p.grid != total * (cta + 1) / p.grid) {
+      // the piece is in slot 1 of the CTA where the segment began when that CTA
+      // finished an earlier segment first, otherwise in slot 0
+      sl = -1;
+      const uint64_t t0 = globaltimer_ns();
+      uint64_t limit = 0;
+      for (uint32_t spins = 0; sl < 0; ++spins) {
+        for (int s = 0; s < 2 && sl < 0; ++s) {
+          const volatile int* hdr =
+              reinterpret_cast<const volatile int*>(base + (size_t)(2 * cta + s) * PF);
+          if (hdr[0] == seg && hdr[3] == tag) sl = s;
+        }
+        if (sl < 0 && (spins & 63u) == 63u) {
+          if (*abort_flag) break;
+          if (limit == 0) limit = wait_limit_ns(p.err);
+          if (globaltimer_ns() - t0 > limit || spins >= kWaitMaxPolls) {
+            record_error(p.err, kDevTimeoutMbarrier);
+            *abort_flag = 1;
+            break;
           }
         }
-        __threadfence();  // the piece's data, published before its header, is read below
-        *found_slot = sl;
       }
-      named_bar_sync(1, NW * 32);
-      slot = *found_slot;
-      named_bar_sync(1, NW * 32);
-      if (slot < 0) return;  // gave up (error recorded)
+      __threadfence();  // the piece's data, published before its header, is read below
     }
-    if (act) absorb(base + (size_t)(2 * cta + slot) * PF + kPartHeader + g * PHF);
+    slots[k] = sl;
   }
-  if (act) write_result<T, D, MODE>(p, b, h0 + g, c, M, L, Z, O, U);
+  named_bar_sync(1, NW * 32);
+  if (tid >= HPW * D) return;
+  const int g = tid / D, c = tid % D;
+  float M = -INFINITY, L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
+  auto absorb = [&](float m, float l, float z, float o, float u) {
+    const float Mn = fmaxf(M, m);
+    const float wa = merge_weight(M, Mn), wb = merge_weight(m, Mn);
+    L = L * wa + l * wb;
+    Z = Z * wa + z * wb;
+    O = O * wa + o * wb;
+    U = U * wa + u * wb;
+    M = Mn;
+  };
+  bool failed = false;
+  // pieces in CTA order, four loads in flight at a time
+  for (int k0 = 0; k0 <= npieces; k0 += 4) {
+    float v[4][5];
+    bool use[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int k = k0 + q;
+      use[q] = false;
+      if (k > npieces) continue;
+      const int sl = k < npieces ? slots[k] : 0;  // k == npieces: this CTA's own piece
+      if (sl == -1) failed = true;
+      if (sl < 0) continue;
+      const float* ph = base + (size_t)(2 * ((int)cf + k) + sl) * PF + kPartHeader + g * PHF;
+      v[q][0] = __ldcg(ph);
+      v[q][1] = __ldcg(ph + 1);
+      v[q][2] = __ldcg(ph + 2);
+      v[q][3] = __ldcg(ph + 4 + c);
+      v[q][4] = __ldcg(ph + 4 + D + c);
+      use[q] = true;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (use[q]) absorb(v[q][0], v[q][1], v[q][2], v[q][3], v[q][4]);
+  }
+  if (!failed) write_result<T, D, MODE>(p, b, h0 + g, c, M, L, Z, O, U);
 }
 
 // ---------------------------------------------------------------------------
@@ -370,7 +391,6 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
   RangeInfo* info = reinterpret_cast<RangeInfo*>(empty + STAGES);
   long long* scan_ws = reinterpret_cast<long long*>(info + 1);   // 16 entries
   volatile int* abort_flag = reinterpret_cast<volatile int*>(scan_ws + 16);
-  int* found_slot = reinterpret_cast<int*>(scan_ws + 18);
   float* merge = reinterpret_cast<float*>(scan_ws + 20);
   float* red_smem = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(merge + NW * HPW * PHF) + 15) & ~uintptr_t(15));
@@ -719,7 +739,7 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     }
     if (done && tail_seg >= 0)
       merge_tail<T, D, HPW, MODE, NW>(p, tail_b, tail_seg, tail_h0, tail_t0, info->total, tid,
-                                      abort_flag, found_slot);
+                                      abort_flag, reinterpret_cast<int*>(merge));
   } else {
     // ------------------------------------------------------------ consumers (fp32)
     const int hw = lane >> 4, sub = lane & 15;
@@ -952,7 +972,7 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     }
     if (done && tail_seg >= 0)
       merge_tail<T, D, HPW, MODE, NW>(p, tail_b, tail_seg, tail_h0, tail_t0, info->total, tid,
-                                      abort_flag, found_slot);
+                                      abort_flag, reinterpret_cast<int*>(merge));
   }
 }
 
@@ -1016,6 +1036,11 @@ constexpr int decode_smem_bytes(int hpw) {
          (Cfg::MMA ? 0 : (2 * Cfg::NW * kDecRedRegion + 2 * Cfg::NW * 16) * 4);
 }
 static_assert(decode_smem_bytes<__nv_bfloat16, 128>(2) <= 227 * 1024, "shared memory");
+// the merge buffer doubles as the piece-slot scratch of merge_tail (one int per
+// CTA of the grid, at most one CTA per SM; 1024 SMs would still fit)
+static_assert(DecodeTile<__nv_bfloat16, 64>::NW * part_head_floats<64>() >= 1024 &&
+                  DecodeTile<float, 64>::NW * part_head_floats<64>() >= 1024,
+              "merge buffer as slot scratch");
 static_assert(decode_smem_bytes<__nv_bfloat16, 64>(2) <= 227 * 1024, "shared memory");
 static_assert(decode_smem_bytes<float, 128>(2) <= 227 * 1024, "shared memory");
 static_assert(decode_smem_bytes<float, 64>(2) <= 227 * 1024, "shared memory");

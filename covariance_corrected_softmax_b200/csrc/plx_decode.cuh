@@ -112,10 +112,6 @@ struct DecodeParams {
   // state over this cache -- m (log2 units of the scaled scores), l, z, 0,
   // o[D], u[D], unnormalised -- is written to state[(b * Hq + h) * (2D + 4)].
   float* state;
-  // Tag of this call (a host-side counter): a split segment's published
-  // pieces carry it, so a piece left in the workspace by an earlier call is
-  // never mistaken for this call's.
-  int call_tag;
 };
 
 // Tile metadata written by the producer next to each stage.

@@ -35,6 +35,15 @@ __device__ __forceinline__ void record_error(unsigned* err, unsigned code) {
   if (err) atomicCAS(err, 0u, code);
 }
 
+// This launch's grid identifier (unique per launch in the context, graph
+// replays included): tags data one launch leaves for another CTA of the same
+// launch, so that what an earlier launch left behind is never mistaken for it.
+__device__ __forceinline__ int launch_tag() {
+  uint64_t id;
+  asm volatile("mov.u64 %0, %%gridid;" : "=l"(id));
+  return (int)((id ^ (id >> 31)) & 0x7fffffffu);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -182,6 +182,35 @@ def test_decode_lengths_far_below_capacity(lens):
     assert torch.equal(out, f32.to(torch.bfloat16))
 
 
+def test_decode_in_a_cuda_graph_replays_with_new_data():
+    """plx_decode captured once in a CUDA graph and replayed after the cache
+    changed: every replay must equal an eager call on the new contents (split
+    segments' pieces carry the launch's identity, so a replay never merges a
+    piece an earlier replay left in the workspace)."""
+    shape = W.DecodeShape(B=6, Hq=16, Hkv=8, d=128, S_max=2000, ctx=2000, ragged=True)
+    inp = W.make_decode(shape, seed=12, device=DEV)
+    other = W.make_decode(shape, seed=13, device=DEV)
+    ws = plx.decode_workspace(shape.B, shape.Hq, shape.Hkv, shape.d, shape.S_max, device=DEV)
+    out = torch.empty_like(inp["q"])
+    args = (inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["seqlens"])
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        plx.decode(*args, softmax_scale=1.0, out=out, workspace=ws)  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        plx.decode(*args, softmax_scale=1.0, out=out, workspace=ws)
+    for src in (other, inp, other):
+        inp["k_cache"].copy_(src["k_cache"])
+        inp["v_cache"].copy_(src["v_cache"])
+        graph.replay()
+        torch.cuda.synchronize()
+        eager = plx.decode(*args, softmax_scale=1.0)
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+
+
 def test_decode_deterministic():
     shape = W.DecodeShape(B=8, Hq=16, Hkv=8, d=128, S_max=3000, ctx=3000, ragged=True)
     inp = W.make_decode(shape, seed=4, device=DEV)
