@@ -225,13 +225,14 @@ def bench_decode(plx, W, shape, steps, warmup, world, device, rank):
 def bench_decode_e2e(plx, W, shape, steps, warmup, world, device, rank):
     """Same metric through the public serving call with host I/O every step: the
     new token's q, rho, k, v and the lengths (which count the new token) are
-    packed in one pinned host buffer and copied host -> device in one copy;
-    plx_decode_append writes k, v into the cache and decodes; out comes back to
-    pinned host memory.  As a serving loop would, the copies run on their own
-    stream, double-buffered: step i+1's inputs go up while step i decodes, and
-    step i's output comes down while step i+1 decodes (every step still moves
-    its own inputs and output).  The time runs from the first copy to the last
-    output landing in host memory."""
+    packed in one pinned host buffer and copied host -> device; plx_decode_append
+    writes k, v into the cache and decodes; out comes back to pinned host
+    memory.  As a serving loop would run it, one step is one replay of a CUDA
+    graph captured from those calls, with the copies on side branches of the
+    graph: step i's graph decodes step i while it uploads step i+1's inputs and
+    downloads step i-1's output (double-buffered; every step still moves its own
+    inputs and output).  The time runs from the first upload to the last output
+    landing in host memory."""
     import torch
     inp = W.make_decode(shape, seed=100 + rank, device=device, copies=3)
     B, Hq, Hkv, d = shape.B, shape.Hq, shape.Hkv, shape.d
@@ -258,44 +259,62 @@ def bench_decode_e2e(plx, W, shape, steps, warmup, world, device, rank):
         outs_h.append(torch.empty((B, Hq, d), dtype=inp["q"].dtype).pin_memory())
         outs_d.append(torch.empty_like(inp["q"]))
     ws = plx.decode_workspace(B, Hq, Hkv, d, shape.S_max, device=device)
-    comp = torch.cuda.current_stream()
-    copy = torch.cuda.Stream(device=device)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
+    cap = torch.cuda.Stream(device=device)
+    s_in = torch.cuda.Stream(device=device)
+    s_out = torch.cuda.Stream(device=device)
 
-    def step(i):
-        b = i % 2
-        v = views[b]
-        with torch.cuda.stream(copy):
-            if i >= 2:
-                copy.wait_event(ev_done[b])  # step i-2 has finished reading this buffer
-            dbufs[b].copy_(hbufs[b], non_blocking=True)
-            ev_in[b].record(copy)
-        comp.wait_event(ev_in[b])
-        if i >= 2:
-            comp.wait_event(ev_out[b])  # step i-2's output has left this buffer
-        plx.decode_append(v["q"], v["rho"], v["k"], v["v"], inp["k_caches"][i % 3],
-                          inp["v_caches"][i % 3], v["sl"], softmax_scale=1.0, out=outs_d[b],
-                          workspace=ws, stream=comp)
-        ev_done[b].record(comp)
-        with torch.cuda.stream(copy):
-            copy.wait_event(ev_done[b])
-            outs_h[b].copy_(outs_d[b], non_blocking=True)
-            ev_out[b].record(copy)
+    def serve(pb, c, stream):
+        v = views[pb]
+        plx.decode_append(v["q"], v["rho"], v["k"], v["v"], inp["k_caches"][c],
+                          inp["v_caches"][c], v["sl"], softmax_scale=1.0, out=outs_d[pb],
+                          workspace=ws, stream=stream)
 
-    for i in range(warmup):
-        step(i)
+    # warm up outside capture (first-call set-up of the library, the allocator)
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        for pb in range(2):
+            dbufs[pb].copy_(hbufs[pb], non_blocking=True)
+            serve(pb, 0, cap)
+            outs_h[pb].copy_(outs_d[pb], non_blocking=True)
+    torch.cuda.synchronize()
+
+    graphs = {}
+    for pb in range(2):          # parity of the step (which I/O buffers)
+        for c in range(3):       # which of the three rotating caches
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                fork = torch.cuda.Event()
+                fork.record(cap)
+                s_in.wait_event(fork)
+                s_out.wait_event(fork)
+                with torch.cuda.stream(s_in):    # the next step's inputs
+                    dbufs[1 - pb].copy_(hbufs[1 - pb], non_blocking=True)
+                with torch.cuda.stream(s_out):   # the previous step's output
+                    outs_h[1 - pb].copy_(outs_d[1 - pb], non_blocking=True)
+                serve(pb, c, cap)                # this step
+                cap.wait_stream(s_in)
+                cap.wait_stream(s_out)
+            graphs[(pb, c)] = g
+    main = torch.cuda.current_stream()
+
+    def run(n, first):
+        dbufs[first % 2].copy_(hbufs[first % 2], non_blocking=True)  # the first step's inputs
+        for i in range(first, first + n):
+            graphs[(i % 2, i % 3)].replay()
+        last = (first + n - 1) % 2
+        outs_h[last].copy_(outs_d[last], non_blocking=True)          # the last step's output
+
+    run(warmup, 0)
     torch.cuda.synchronize()
     barrier(world)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(copy)
-    for i in range(steps):
-        step(warmup + i)
-    e.record(copy)  # after the last output's copy to the host
+    s.record(main)
+    run(steps, warmup)
+    e.record(main)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world, device)
+    del graphs
     h2d = hbufs[0].numel()
     d2h = outs_h[0].numel() * outs_h[0].element_size()
     return {"ms": ms, "h2d": h2d, "d2h": d2h}
@@ -426,7 +445,9 @@ def prefill_record(name, pshape, pr, psteps, world, peaks, peak_src, traffic):
                      "peak_sustained": peaks["bf16_tflops_sustained"],
                      "frac_sustained": tflops / peaks["bf16_tflops_sustained"],
                      "flops_per_call": pshape.flops(), "traffic": traffic},
-        "gpu_launches_per_call": 1,
+        # the fast instance and the recomputing one (which returns at once
+        # when no unit's V is out of fp16's range)
+        "gpu_launches_per_call": 2,
         "clocks": pr["clocks"],
     }
 
@@ -539,8 +560,9 @@ def main():
                    "unit": "tokens/s",
                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                    "ms_per_step": e2e["ms"] / args.steps,
-                   "call": "plx_decode_append (KV append + decode)",
-                   "gpu_launches": 3 * args.steps}
+                   "call": "plx_decode_append (KV append + decode), one CUDA-graph replay per "
+                           "step with the copies of the neighbouring steps on side branches",
+                   "gpu_launches": 2 * args.steps}
 
     prefill = prefill_long = None
     if not args.no_prefill:
@@ -582,12 +604,12 @@ def main():
         "hbm_gbs": gbs,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"],
-                     "kernel": "plx_decode (split-K main kernel + combine kernel)",
+                     "kernel": "plx_decode (one persistent split-K kernel, merge included)",
                      "peak_source": f"{peak_src} HBM copy bandwidth",
                      "bytes_per_call": dec["alg_bytes"], "traffic": traffic},
         "cpu_baseline": cpu,
         "e2e": e2e_rec,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": args.steps,
         "clocks": dec["clocks"],
         "prefill": prefill,
         "prefill_long": prefill_long,
