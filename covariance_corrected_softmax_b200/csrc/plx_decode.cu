@@ -217,11 +217,14 @@ __device__ __forceinline__ void write_result(const DecodeParams& p, int b, int h
 //    segment) is merged with the earlier pieces once the CTA has finished all
 //    its tiles (merge_tail below): every CTA holds about the same work, so the
 //    CTAs holding those pieces finish at about the same time.
-// Called by all consumer threads between two consumer-wide barriers.
+// Called by all consumer threads between two consumer-wide barriers; false if
+// the consumer barrier (cbar) gave up.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int HPW, int MODE, int NW>
-__device__ __forceinline__ void finalize_segment(const DecodeParams& p, const TileMeta& mt, int h0,
-                                                 float* part, const float* merge, int tid) {
+__device__ __forceinline__ bool finalize_segment(const DecodeParams& p, const TileMeta& mt, int h0,
+                                                 float* part, const float* merge, int tid,
+                                                 uint64_t* cbar, uint32_t& cphase,
+                                                 volatile int* abort_flag) {
   constexpr int PHF = part_head_floats<D>();
   static_assert(HPW * D <= NW * 32, "one element per consumer thread");
   const bool starts = (mt.flags & 4) != 0, ends = (mt.flags & 8) != 0;
@@ -256,7 +259,7 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams& p, const Ti
   if (!ends) {
     // publish: the data above, then the header
     __threadfence();
-    named_bar_sync(1, NW * 32);
+    if (!warps_sync(cbar, cphase, abort_flag, p.err)) return false;
     if (tid == 0) {
       volatile int* hdr = reinterpret_cast<volatile int*>(part);
       hdr[1] = starts ? 1 : 0;
@@ -266,6 +269,7 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams& p, const Ti
       hdr[0] = mt.seg;
     }
   }
+  return true;
 }
 
 // The split segment whose last piece this CTA holds (in its slot 0): merge the
@@ -278,7 +282,8 @@ __device__ __forceinline__ void finalize_segment(const DecodeParams& p, const Ti
 template <typename T, int D, int HPW, int MODE, int NW>
 __device__ __forceinline__ void merge_tail(const DecodeParams& p, int b, int seg, int h0,
                                            long long seg_t0, long long total, int tid,
-                                           volatile int* abort_flag, int* slots) {
+                                           volatile int* abort_flag, int* slots, uint64_t* cbar,
+                                           uint32_t& cphase) {
   constexpr int PF = part_floats<D>(HPW);
   constexpr int PHF = part_head_floats<D>();
   const float* base = p.ws + kWsHeaderFloats;
@@ -316,7 +321,7 @@ __device__ __forceinline__ void merge_tail(const DecodeParams& p, int b, int seg
     }
     slots[k] = sl;
   }
-  named_bar_sync(1, NW * 32);
+  if (!warps_sync(cbar, cphase, abort_flag, p.err)) return;
   if (tid >= HPW * D) return;
   const int g = tid / D, c = tid % D;
   float M = -INFINITY, L = 0.f, Z = 0.f, O = 0.f, U = 0.f;
@@ -391,6 +396,7 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
   RangeInfo* info = reinterpret_cast<RangeInfo*>(empty + STAGES);
   long long* scan_ws = reinterpret_cast<long long*>(info + 1);   // 16 entries
   volatile int* abort_flag = reinterpret_cast<volatile int*>(scan_ws + 16);
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(scan_ws + 18);  // the consumer warps' barrier
   float* merge = reinterpret_cast<float*>(scan_ws + 20);
   float* red_smem = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(merge + NW * HPW * PHF) + 15) & ~uintptr_t(15));
@@ -404,6 +410,7 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NW);
     }
+    mbar_init(cbar, NW);
     fence_mbarrier_init();
   }
   locate_range(p, TK, info, scan_ws);  // contains __syncthreads
@@ -560,6 +567,7 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     int tail_seg = -1, tail_b = 0, tail_h0 = 0;  // the split segment ending here
     long long tail_t0 = 0;
     bool done = true;
+    uint32_t cphase = 0;  // completed uses of the consumer barrier
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
@@ -722,12 +730,16 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
         }
       }
       if (mt.flags & 2) {
-        named_bar_sync(1, NW * 32);
         // slot 0 holds the CTA's first segment, which may have begun in an
         // earlier CTA; slot 1 its last, which may end in a later one
         float* part = p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + (ordinal == 0 ? 0 : 1)) * PF;
-        finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, part, merge, tid);
-        named_bar_sync(1, NW * 32);
+        if (!warps_sync(cbar, cphase, abort_flag, p.err) ||
+            !finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, part, merge, tid, cbar, cphase,
+                                                   abort_flag) ||
+            !warps_sync(cbar, cphase, abort_flag, p.err)) {
+          done = false;
+          break;
+        }
         if ((mt.flags & 8) && !(mt.flags & 4)) {  // this CTA holds a split segment's end
           tail_seg = mt.seg;
           tail_b = mt.b;
@@ -739,7 +751,7 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     }
     if (done && tail_seg >= 0)
       merge_tail<T, D, HPW, MODE, NW>(p, tail_b, tail_seg, tail_h0, tail_t0, info->total, tid,
-                                      abort_flag, reinterpret_cast<int*>(merge));
+                                      abort_flag, reinterpret_cast<int*>(merge), cbar, cphase);
   } else {
     // ------------------------------------------------------------ consumers (fp32)
     const int hw = lane >> 4, sub = lane & 15;
@@ -765,6 +777,7 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     int tail_seg = -1, tail_b = 0, tail_h0 = 0;  // the split segment ending here
     long long tail_t0 = 0;
     bool done = true;
+    uint32_t cphase = 0;  // completed uses of the consumer barrier
 #pragma unroll
     for (int g = 0; g < HPW; ++g) {
 #pragma unroll
@@ -957,10 +970,14 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
             }
           }
         }
-        named_bar_sync(1, NW * 32);
         float* part = p.ws + kWsHeaderFloats + (size_t)(2 * blockIdx.x + (ordinal == 0 ? 0 : 1)) * PF;
-        finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, part, merge, tid);
-        named_bar_sync(1, NW * 32);
+        if (!warps_sync(cbar, cphase, abort_flag, p.err) ||
+            !finalize_segment<T, D, HPW, MODE, NW>(p, mt, h0, part, merge, tid, cbar, cphase,
+                                                   abort_flag) ||
+            !warps_sync(cbar, cphase, abort_flag, p.err)) {
+          done = false;
+          break;
+        }
         if ((mt.flags & 8) && !(mt.flags & 4)) {  // this CTA holds a split segment's end
           tail_seg = mt.seg;
           tail_b = mt.b;
@@ -972,7 +989,7 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
     }
     if (done && tail_seg >= 0)
       merge_tail<T, D, HPW, MODE, NW>(p, tail_b, tail_seg, tail_h0, tail_t0, info->total, tid,
-                                      abort_flag, reinterpret_cast<int*>(merge));
+                                      abort_flag, reinterpret_cast<int*>(merge), cbar, cphase);
   }
 }
 

@@ -198,6 +198,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return true;
 }
 
+// A barrier among whole warps on an mbarrier initialised with their number (one
+// arrival per warp), bounded like mbar_wait: false in every lane of the warp if
+// the wait gave up (a warp that left its loop early never arrives, so the
+// others record a timeout instead of waiting for good).  `phase` counts the
+// caller's completed uses of the barrier.
+__device__ __forceinline__ bool warps_sync(uint64_t* bar, uint32_t& phase, volatile int* abort,
+                                           unsigned* err) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase & 1u, abort, err);
+  ++phase;
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), plain tile loads into this CTA's
 // shared memory, completing on an mbarrier with a transaction count.
@@ -414,6 +428,21 @@ __device__ __forceinline__ void tmem_wait_st() {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier that also ORs a predicate over the participating threads: every
+// thread gets the same answer, so a group can leave a loop together.
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "barrier.cta.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ---------------------------------------------------------------------------
