@@ -698,6 +698,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool qpos = p.qscale >= 0.f;
     int g = 0, xs = 0, uc = 0;  // uc: units with work so far
     bool ok = true, finite = true;
+    // A wait of this thread gave up (sticky).  The thread carries on through
+    // the same steps (its TMEM and memory accesses stay in bounds; the values
+    // no longer matter) and passes the flag to its partner with the partial
+    // maxima, as a negative max |t|: both threads of the row leave at the same
+    // exchange, so neither is left waiting at the named barrier.
+    bool failed = false;
     for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
       const Unit x = unit_at<VARLEN, SAFE>(p, u, umask);
       if (x.n == 0) continue;  // (varlen) no such query tile
@@ -742,14 +748,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int j = 0; j < x.n; ++j) {
         const int t = g + j;
-        if (SAFE && j > 0 && !v_check(t - 1, j - 1)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait(&bars->s_full, t & 1, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
+        if (SAFE && j > 0 && !v_check(t - 1, j - 1)) failed = true;
+        if (!mbar_wait(&bars->s_full, t & 1, abort_flag, p.err)) failed = true;
         tc_fence_after();
         uint32_t sv[kHalf], tv[kHalf];
         tmem_ld2x32_sync(lane_addr + C::COL_S + my_cols, lane_addr + C::COL_T + my_cols, sv, tv);
@@ -789,10 +789,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         float part_max = (nvis > 0) ? ext * p.qscale : -INFINITY;
         float tmax = fmaxf(t2[0], t2[1]);
         // combine with the partner half of the row
-        xch->tile[xs & 1][half][r] = make_float2(part_max, tmax);
+        xch->tile[xs & 1][half][r] = make_float2(part_max, failed ? -1.f : tmax);
         named_bar_sync(bar_id, 64);
         {
           const float2 o = xch->tile[xs & 1][half ^ 1][r];
+          if (failed || o.y < 0.f) {
+            ok = false;
+            break;
+          }
           part_max = fmaxf(part_max, o.x);
           tmax = fmaxf(tmax, o.y);
         }
@@ -847,10 +851,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // the P columns (and O, U) are free once the previous tile's PV has completed
-        if (j > 0 && !mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, p.err)) {
-          ok = false;
-          break;
-        }
+        if (j > 0 && !mbar_wait(&bars->o_done, (t - 1) & 1, abort_flag, p.err)) failed = true;
         tc_fence_after();
         tmem_st16(lane_addr + C::COL_P + my_cols / 2, pk);
         // P t 2^-eu as fp16 pairs
@@ -895,7 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: out = ((1 + z/l) o - u) / l, lse = ln(sum exp(scale s));
       // l and z are the ones-columns of O and U; each half writes half the row.
       const int tl = g + x.n - 1;
-      if (SAFE && !v_check(tl, x.n - 1)) break;
+      if (SAFE && !v_check(tl, x.n - 1)) failed = true;
       bool oor = false;  // fast instance: this unit's V is out of range (marker)
       if constexpr (!SAFE) {
         // posted by the converters with the unit count once the unit's last V
@@ -915,16 +916,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             w = *tag;
           }
-          if ((int)(uint32_t)w != uc) {
-            ok = false;
-            break;
-          }
+          if ((int)(uint32_t)w != uc) failed = true;
           oor = oor || (w >> 32) != 0;
         }
-        if (!ok) break;
         ++uc;
       }
-      if (!mbar_wait(&bars->o_done, tl & 1, abort_flag, p.err)) break;
+      if (!mbar_wait(&bars->o_done, tl & 1, abort_flag, p.err)) failed = true;
       tc_fence_after();
       uint32_t lw, zw;
       tmem_ld2x1_sync(lane_addr + C::COL_O + D, lane_addr + C::COL_U + D, lw, zw);
