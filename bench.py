@@ -524,6 +524,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["plx", "reference"], default="plx")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-prefill-long", action="store_true",
+                    help="skip the long-context prefill leg (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-I/O leg (profiling)")
     ap.add_argument("--no-sweep", action="store_true", help="skip the decode grid")
@@ -566,7 +568,8 @@ def main():
 
     prefill = prefill_long = None
     if not args.no_prefill:
-        for name, psteps in ((PREFILL, 40), (PREFILL_LONG, 8)):
+        legs = ((PREFILL, 40),) if args.no_prefill_long else ((PREFILL, 40), (PREFILL_LONG, 8))
+        for name, psteps in legs:
             pshape = W.WORKLOADS[name]
             pr = bench_prefill(plx, W, pshape, psteps, 3, world, device, rank)
             if "ms" in pr:
