@@ -586,9 +586,14 @@ plx_status plx_prefill_bwd(const void* q, const void* rho, const void* k, const 
   if ((long long)B * L * H_q > 0x7fffffffll * 8) return PLX_ERR_UNSUPPORTED;
   if (workspace_bytes < plx::prefill_bwd_workspace_bytes(B, L, H_q))
     return PLX_ERR_WORKSPACE_TOO_SMALL;
-  const cudaError_t e = plx::launch_prefill_bwd(q, rho, k, v, dout, dq, drho, dk, dv, workspace,
-                                                causal, B, L, H_q, H_kv, d, dtype == PLX_BF16,
-                                                softmax_scale, static_cast<cudaStream_t>(stream));
+  int sms = 0;
+  unsigned* err = nullptr;
+  cudaError_t e = device_info(&sms, &err);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = plx::launch_prefill_bwd(q, rho, k, v, dout, dq, drho, dk, dv, workspace, causal, B, L, H_q,
+                              H_kv, d, dtype == PLX_BF16, softmax_scale, err, sms,
+                              static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return PLX_ERR_UNSUPPORTED;
   return e == cudaSuccess ? PLX_OK : cuda_fail(e);
 }
 

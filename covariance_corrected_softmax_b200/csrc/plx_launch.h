@@ -67,13 +67,29 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache
 cudaError_t launch_probe_projection(const void* x, const void* w, void* rho, int M, int N, int K,
                                     bool bf16, int num_sms, unsigned* err, cudaStream_t stream);
 
-// Gradients of the prefill operator (CUDA cores): dq, drho [B, L, Hq, d],
-// dk, dv [B, L, Hkv, d], all fp32; workspace of prefill_bwd_workspace_bytes().
+// Gradients of the prefill operator: dq, drho [B, L, Hq, d], dk, dv
+// [B, L, Hkv, d], all fp32; workspace of prefill_bwd_workspace_bytes().  fp32
+// inputs run on the CUDA cores, bf16 inputs on the tensor cores (below).
 size_t prefill_bwd_workspace_bytes(int B, int L, int Hq);
 cudaError_t launch_prefill_bwd(const void* q, const void* rho, const void* k, const void* v,
                                const void* dout, float* dq, float* drho, float* dk, float* dv,
                                void* workspace, int causal, int B, int L, int Hq, int Hkv, int d,
-                               bool bf16, float scale, cudaStream_t stream);
+                               bool bf16, float scale, unsigned* err, int num_sms,
+                               cudaStream_t stream);
+
+// The same gradients for bf16 inputs on the tensor cores (two tcgen05 kernels;
+// d = 64 or 128).  The workspace holds the row statistics the first kernel
+// computes for the second.
+struct BwdTcArgs {
+  const void *q, *rho, *k, *v, *dout;  // bf16
+  float *dq, *drho, *dk, *dv;
+  void* workspace;  // prefill_bwd_workspace_bytes()
+  int B, L, Hq, Hkv, d, causal;
+  float scale;
+  unsigned* err;
+  int num_sms;
+};
+cudaError_t launch_prefill_bwd_tc(const BwdTcArgs& a, cudaStream_t stream);
 
 // One warp that waits on an mbarrier nothing ever completes, with the
 // device's bounded wait: it records kDevTimeoutMbarrier when the limit runs out

@@ -1,5 +1,7 @@
-// plx_prefill_bwd.cu -- gradients of the Parallax prefill operator (CUDA
-// cores, fp32 arithmetic for fp32 and bf16 inputs).
+// plx_prefill_bwd.cu -- gradients of the Parallax prefill operator for fp32
+// inputs (CUDA cores, fp32 arithmetic throughout: the fp32 bar needs fp32
+// products).  bf16 inputs go to the tensor-core kernels of
+// plx_prefill_bwd_tc.cu.
 //
 // Operator (page 1 "Parallax: Parameterized Local Linear Attention Gives
 // Transformers a 'Second Eye'", opening formula and section 1.3; page 3
@@ -234,7 +236,32 @@ size_t prefill_bwd_workspace_bytes(int B, int L, int Hq) {
 cudaError_t launch_prefill_bwd(const void* q, const void* rho, const void* k, const void* v,
                                const void* dout, float* dq, float* drho, float* dk, float* dv,
                                void* workspace, int causal, int B, int L, int Hq, int Hkv, int d,
-                               bool bf16, float scale, cudaStream_t stream) {
+                               bool bf16, float scale, unsigned* err, int num_sms,
+                               cudaStream_t stream) {
+  if (bf16) {
+    // bf16: the tensor-core kernels
+    BwdTcArgs a;
+    a.q = q;
+    a.rho = rho;
+    a.k = k;
+    a.v = v;
+    a.dout = dout;
+    a.dq = dq;
+    a.drho = drho;
+    a.dk = dk;
+    a.dv = dv;
+    a.workspace = workspace;
+    a.B = B;
+    a.L = L;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.d = d;
+    a.causal = causal;
+    a.scale = scale;
+    a.err = err;
+    a.num_sms = num_sms;
+    return launch_prefill_bwd_tc(a, stream);
+  }
   BwdParams p;
   p.q = q;
   p.rho = rho;
@@ -253,13 +280,8 @@ cudaError_t launch_prefill_bwd(const void* q, const void* rho, const void* k, co
   p.G = Hq / Hkv;
   p.causal = causal;
   p.scale = scale;
-  if (bf16) {
-    if (d == 128) return launch_bwd_t<__nv_bfloat16, 128>(p, stream);
-    if (d == 64) return launch_bwd_t<__nv_bfloat16, 64>(p, stream);
-  } else {
-    if (d == 128) return launch_bwd_t<float, 128>(p, stream);
-    if (d == 64) return launch_bwd_t<float, 64>(p, stream);
-  }
+  if (d == 128) return launch_bwd_t<float, 128>(p, stream);
+  if (d == 64) return launch_bwd_t<float, 64>(p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -65,3 +65,26 @@ def test_bwd_bf16_l1024_outlier_keys(causal):
     shape = W.PrefillShape(B=1, L=1024, Hq=4, Hkv=2, d=128, outlier_frac=0.01, causal=causal)
     inp = W.make_prefill(shape, seed=5, device=DEV)
     _compare(inp, _dout(inp["q"].shape, 3, torch.bfloat16), causal, 1.0, True, "bf16 L=1024")
+
+
+BF16_CASES = [(1, 1, 2, 1, 64, True), (1, 65, 4, 2, 64, True), (2, 200, 2, 1, 128, False),
+              (1, 300, 3, 3, 128, True), (1, 520, 4, 2, 128, True), (2, 129, 2, 2, 64, False)]
+
+
+@pytest.mark.parametrize("case", BF16_CASES, ids=[f"b{i}" for i in range(len(BF16_CASES))])
+def test_bwd_bf16_shapes(case):
+    """bf16 inputs (the tensor-core kernels) over ragged lengths that span
+    several 64- and 128-row tiles and their partial tails, GQA groups of 1-2,
+    d = 64 and 128, causal and not: every gradient at the bf16 bar."""
+    B, L, Hq, Hkv, d, causal = case
+    shape = W.PrefillShape(B=B, L=L, Hq=Hq, Hkv=Hkv, d=d, rho_std=0.3)
+    inp = W.make_prefill(shape, seed=7 * L + d, device=DEV)
+    _compare(inp, _dout(inp["q"].shape, 4, torch.bfloat16), causal, 1.0 / np.sqrt(d), True,
+             str(case))
+
+
+def test_bwd_bf16_negative_scale():
+    """A negative softmax scale (the softmax favours the smallest scores)."""
+    shape = W.PrefillShape(B=1, L=257, Hq=2, Hkv=1, d=128, rho_std=0.3)
+    inp = W.make_prefill(shape, seed=11, device=DEV)
+    _compare(inp, _dout(inp["q"].shape, 5, torch.bfloat16), True, -0.2, True, "negative scale")
