@@ -7,7 +7,9 @@ H_kv=8, d=128, context 4096 (``decode_b32_ctx4096``).  One step is one
 split merge).  The causal prefill rows of the hot path are measured in the same
 run on ``prefill_b8_l4096`` (B=8, L=4096, H_q=16, H_kv=8, d=128) and reported
 under ``"prefill"``, the long-context prefill ``prefill_b1_l32768`` (B=1,
-L=32768, H_q=32, H_kv=8) under ``"prefill_long"``, and the decode grid (batch
+L=32768, H_q=32, H_kv=8) under ``"prefill_long"``, the gradients of the prefill
+(``plx_prefill_bwd`` on ``prefill_b8_l4096``, 16d flops per visible pair) under
+``"prefill_bwd"``, and the decode grid (batch
 1-2048 x context 128-32768, ragged lengths) under ``"sweep"``: per cell the
 device time per call with L2 flushed before every call, HBM GB/s from the
 actual lengths and the fraction of the measured copy bandwidth.
@@ -381,6 +383,68 @@ def bench_prefill(plx, W, shape, steps, warmup, world, device, rank):
     return {"ms": ms, "clocks": clk.summary()}
 
 
+def bench_prefill_bwd(plx, W, shape, steps, warmup, world, device, rank):
+    """plx_prefill_bwd (bf16: the two tensor-core kernels) on the prefill
+    workload with a seeded dout; the gradients and the statistics workspace are
+    allocated once, outside the timed region."""
+    import torch
+    x = W.make_prefill(shape, seed=40 + rank, device=device)
+    g = torch.Generator(device=device).manual_seed(41 + rank)
+    dout = torch.randn(x["q"].shape, generator=g, device=device).to(x["q"].dtype)
+    grads = [torch.empty(x[n].shape, dtype=torch.float32, device=device)
+             for n in ("q", "rho", "k", "v")]
+    ws = torch.empty(plx.prefill_bwd_workspace_bytes(shape.B, shape.L, shape.Hq),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        plx.prefill_bwd(x["q"], x["rho"], x["k"], x["v"], dout, causal=shape.causal,
+                        softmax_scale=1.0, grads=grads, workspace=ws, stream=stream)
+
+    try:
+        step()
+    except plx.PlxError as e:
+        return {"status": str(e)}
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_index()) as clk:
+        s.record(stream)
+        for _ in range(steps):
+            step()
+        e.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world, device)
+    assert plx.device_error() == 0, "backward kernels reported a device error"
+    return {"ms": ms, "clocks": clk.summary()}
+
+
+def prefill_bwd_record(name, pshape, pr, psteps, peaks, peak_src):
+    pms = pr["ms"] / psteps
+    # 16d flops per visible (query, key) pair: the eight products S, T, GV,
+    # dV, dQ, dR and the two of dK, each 2d per pair (recomputation of the row
+    # statistics not counted)
+    flops = 2.0 * pshape.flops()
+    tflops = flops / (pms / 1e3) / 1e12
+    return {
+        "workload": name, "B": pshape.B, "L": pshape.L, "H_q": pshape.Hq, "H_kv": pshape.Hkv,
+        "d": pshape.d, "causal": pshape.causal, "steps": psteps, "ms_per_call": pms,
+        "tflops": tflops,
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "peak_sustained": peaks["bf16_tflops_sustained"],
+                     "frac_sustained": tflops / peaks["bf16_tflops_sustained"],
+                     "flops_per_call": flops, "traffic": None},
+        # the rows kernel (dq, drho, row statistics) and the keys kernel (dk, dv)
+        "gpu_launches_per_call": 2,
+        "clocks": pr["clocks"],
+    }
+
+
 # ------------------------------------------------------------------ decode grid
 def bench_decode_sweep(plx, W, peaks, device, only=None):
     """Every cell of the decode grid (batch x context, ragged lengths U[ctx/2,
@@ -526,6 +590,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-prefill-long", action="store_true",
                     help="skip the long-context prefill leg (profiling)")
+    ap.add_argument("--no-prefill-bwd", action="store_true", help="skip the backward leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-I/O leg (profiling)")
     ap.add_argument("--no-sweep", action="store_true", help="skip the decode grid")
@@ -582,6 +647,13 @@ def main():
             else:
                 prefill_long = rec_p
 
+    prefill_bwd = None
+    if not args.no_prefill and not args.no_prefill_bwd:
+        pshape = W.WORKLOADS[PREFILL]
+        pr = bench_prefill_bwd(plx, W, pshape, 10, 3, world, device, rank)
+        prefill_bwd = (prefill_bwd_record(PREFILL, pshape, pr, 10, peaks, peak_src)
+                       if "ms" in pr else {"workload": PREFILL, **pr})
+
     sweep = None
     if not args.no_sweep:
         with ClockSampler(gpu_index()) as clk:
@@ -616,6 +688,7 @@ def main():
         "clocks": dec["clocks"],
         "prefill": prefill,
         "prefill_long": prefill_long,
+        "prefill_bwd": prefill_bwd,
         "sweep": sweep,
     }
     if rank == 0:

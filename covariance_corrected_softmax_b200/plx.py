@@ -254,11 +254,18 @@ def decode_x(q: torch.Tensor, x: torch.Tensor, w_r: torch.Tensor, k_cache: torch
     return out, rho
 
 
+def prefill_bwd_workspace_bytes(B: int, L: int, Hq: int) -> int:
+    return int(lib().plx_prefill_bwd_workspace_bytes(B, L, Hq))
+
+
 def prefill_bwd(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                 dout: torch.Tensor, causal: bool = True, softmax_scale: Optional[float] = None,
+                grads=None, workspace: Optional[torch.Tensor] = None,
                 stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
     """Gradients (dq, drho, dk, dv), fp32, of sum(dout * out) for the forward
-    plx.prefill(q, rho, k, v, causal, softmax_scale)."""
+    plx.prefill(q, rho, k, v, causal, softmax_scale).  `grads` (four fp32
+    tensors shaped like q, rho, k, v) and `workspace` may be passed in to be
+    reused across calls."""
     _same(q, rho, k, v, dout)
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -266,11 +273,19 @@ def prefill_bwd(q: torch.Tensor, rho: torch.Tensor, k: torch.Tensor, v: torch.Te
             v.shape != k.shape:
         raise ValueError("shape mismatch among q, rho, k, v, dout")
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
-    f32 = dict(dtype=torch.float32, device=q.device)
-    dq, drho = torch.empty(q.shape, **f32), torch.empty(q.shape, **f32)
-    dk, dv = torch.empty(k.shape, **f32), torch.empty(k.shape, **f32)
-    nws = int(lib().plx_prefill_bwd_workspace_bytes(B, L, Hq))
-    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=q.device)
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=q.device)
+        dq, drho = torch.empty(q.shape, **f32), torch.empty(q.shape, **f32)
+        dk, dv = torch.empty(k.shape, **f32), torch.empty(k.shape, **f32)
+    else:
+        dq, drho, dk, dv = grads
+        for t_, ref in ((dq, q), (drho, q), (dk, k), (dv, k)):
+            if t_.dtype != torch.float32 or t_.shape != ref.shape or not t_.is_contiguous() or \
+                    t_.device != q.device:
+                raise ValueError("grads must be contiguous fp32 tensors shaped like q, rho, k, v")
+    nws = prefill_bwd_workspace_bytes(B, L, Hq)
+    ws = workspace if workspace is not None else \
+        torch.empty(max(nws, 16), dtype=torch.uint8, device=q.device)
     st = lib().plx_prefill_bwd(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(dout),
                                _ptr(dq), _ptr(drho), _ptr(dk), _ptr(dv), int(bool(causal)), B, L,
                                Hq, Hkv, d, _dtype_code(q), scale, _ptr(ws), ws.numel(),
