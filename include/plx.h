@@ -195,8 +195,10 @@ PLX_API plx_status plx_prefill_fwd_x(const void* q, const void* x, const void* w
  * lse is needed: the kernels recompute what they use, the softmax normaliser
  * included, from q, rho, k, v in fp32 (where one key dominates a row, the
  * gradient's a (X - D) terms cancel and would amplify the fp16 rounding that
- * the tensor-core forward's normaliser carries).  Runs on the CUDA cores with
- * fp32 arithmetic (a correctness path, not tuned).
+ * the tensor-core forward's normaliser carries).  bf16 inputs (d = 64 or 128)
+ * run two tcgen05 kernels (fp32 accumulation; each gradient operand enters the
+ * products as bf16 high and low parts, about 16 significant bits); fp32 inputs
+ * run on the CUDA cores with fp32 arithmetic.  Two launches per call.
  */
 PLX_API size_t plx_prefill_bwd_workspace_bytes(int B, int L, int H_q);
 PLX_API plx_status plx_prefill_bwd(const void* q, const void* rho, const void* k, const void* v,
