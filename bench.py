@@ -450,9 +450,12 @@ def bench_decode_sweep(plx, W, peaks, device, only=None):
     """Every cell of the decode grid (batch x context, ragged lengths U[ctx/2,
     ctx], caches capped under 120e9 bytes).  Each call is timed alone with CUDA
     events, after a 256 MiB buffer (twice the L2) has been written, so every
-    call reads its cache from HBM; the median over the calls is reported."""
+    call reads its cache from HBM, and a second 256 MiB buffer has been read, so
+    that the lines the write left dirty are written back before the timed call
+    rather than during it; the median over the calls is reported."""
     import torch
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    clean = torch.zeros(32 << 20, dtype=torch.int64, device=device)  # 256 MiB
     stream = torch.cuda.current_stream()
     cells = []
     for cell in W.sweep_cells():
@@ -474,6 +477,7 @@ def bench_decode_sweep(plx, W, peaks, device, only=None):
               for _ in range(n)]
         for s_, e_ in ev:
             flush.fill_(1)
+            clean.sum()
             s_.record(stream)
             call()
             e_.record(stream)
@@ -488,7 +492,7 @@ def bench_decode_sweep(plx, W, peaks, device, only=None):
         del inp, ws, out
         torch.cuda.empty_cache()
     assert plx.device_error() == 0, "decode kernels reported a device error in the sweep"
-    del flush
+    del flush, clean
     torch.cuda.empty_cache()
     return cells
 
@@ -660,7 +664,9 @@ def main():
             cells = bench_decode_sweep(plx, W, peaks, device, args.sweep_cells)
         long_ctx = [c for c in cells if c["context"] >= 8192 and not c["launch_bound"]]
         sweep = {"grid": "H_q=16, H_kv=8, d=128, bf16; batch x context, lengths U[ctx/2, ctx]",
-                 "timing": "median of per-call CUDA-event times, 256 MiB L2 flush before each call",
+                 "timing": "median of per-call CUDA-event times; before each call a 256 MiB "
+                           "buffer is written (L2 flush) and another 256 MiB read (dirty "
+                           "lines written back before the call)",
                  "peak": peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy bandwidth",
                  "cells": cells,
                  "min_frac_ctx_ge_8192": min((c["frac"] for c in long_ctx), default=None),
