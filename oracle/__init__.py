@@ -27,7 +27,9 @@ Also here: the probe projection ``rho = W_R x`` (page 1 section 1.3: one extra
 projection matrix; page 3: rho_i = W_R x_i), and the gradients of the prefill
 operator (the pages print none; the derivation is written out in
 ``plx_oracle.c``), pinned by central finite differences of the forward and by
-fp64 autograd of the explicit-covariance definition.
+fp64 autograd of the explicit-covariance definition; ``prefill_bwd_sampled``
+evaluates selected entries of the same gradients in numpy, row by row, and is
+pinned against the C routine.
 """
 from __future__ import annotations
 
@@ -271,6 +273,73 @@ def _streams(k, v, b, hk, n: int):
     vs = np.stack([_f64(v[int(pb), :n, int(ph), :]) for pb, ph in uniq]) if len(uniq) else \
         np.zeros((0, n, v.shape[-1]))
     return inv.reshape(-1), ks, vs
+
+
+def prefill_bwd_sampled(q, rho, k, v, g, causal: bool, scale: float, rows=None, keys=None):
+    """Selected entries of the prefill gradients, fp64, in plain numpy one row
+    at a time (for large shapes, where the full routine would take too long):
+    dq, drho at the query rows ``rows`` [R, 3] of (b, h, i), and dk, dv at the
+    key rows ``keys`` [S, 3] of (b, hk, j).  The operator and its gradients are
+    those of ``plxo_prefill_bwd`` (derivation in ``plx_oracle.c``): for row i
+    with visible keys j, a = softmax(scale q.k), t = rho.k, gv = g.v,
+    tbar = sum a t, go = sum a gv, c = 1 + tbar - t, out = sum a c v,
+    D = g.out + tbar go, ds = a (c gv + t go - D), dt = a (go - gv);
+    dq = scale sum ds k, drho = sum dt k; dk_j = sum over the rows that see key
+    j of scale ds q + dt rho; dv_j = sum a c g.  Returns (dq [R, d], drho [R, d],
+    dk [S, d], dv [S, d])."""
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    streams = {}
+
+    def stream(b, hk):
+        if (b, hk) not in streams:
+            streams[(b, hk)] = (_f64(k[b, :, hk, :]), _f64(v[b, :, hk, :]))
+        return streams[(b, hk)]
+
+    cache = {}
+
+    def row(b, h, i):
+        if (b, h, i) not in cache:
+            K, V = stream(b, h // G)
+            n = i + 1 if causal else L
+            K, V = K[:n], V[:n]
+            qi, ri, gi = _f64(q[b, i, h, :]), _f64(rho[b, i, h, :]), _f64(g[b, i, h, :])
+            s = scale * (K @ qi)
+            a = np.exp(s - s.max())
+            a /= a.sum()
+            t = K @ ri
+            gv = V @ gi
+            tbar = float(a @ t)
+            go = float(a @ gv)
+            c = 1.0 + tbar - t
+            out = (a * c) @ V
+            D = float(gi @ out) + tbar * go
+            ds = a * (c * gv + t * go - D)
+            dt = a * (go - gv)
+            cache[(b, h, i)] = (K, qi, ri, gi, a, c, ds, dt)
+        return cache[(b, h, i)]
+
+    rows = np.zeros((0, 3), dtype=np.int64) if rows is None else \
+        np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+    keys = np.zeros((0, 3), dtype=np.int64) if keys is None else \
+        np.asarray(keys, dtype=np.int64).reshape(-1, 3)
+    dq = np.zeros((len(rows), d))
+    drho = np.zeros((len(rows), d))
+    for r, (b, h, i) in enumerate(rows):
+        K, _, _, _, _, _, ds, dt = row(int(b), int(h), int(i))
+        dq[r] = scale * (ds @ K)
+        drho[r] = dt @ K
+    dk = np.zeros((len(keys), d))
+    dv = np.zeros((len(keys), d))
+    for r, (b, hk, j) in enumerate(keys):
+        b, hk, j = int(b), int(hk), int(j)
+        for h in range(hk * G, (hk + 1) * G):
+            for i in range(j if causal else 0, L):
+                _, qi, ri, gi, a, c, ds, dt = row(b, h, i)
+                dk[r] += scale * ds[j] * qi + dt[j] * ri
+                dv[r] += a[j] * c[j] * gi
+    return dq, drho, dk, dv
 
 
 _default: Optional[Oracle] = None

@@ -88,3 +88,30 @@ def test_bwd_bf16_negative_scale():
     shape = W.PrefillShape(B=1, L=257, Hq=2, Hkv=1, d=128, rho_std=0.3)
     inp = W.make_prefill(shape, seed=11, device=DEV)
     _compare(inp, _dout(inp["q"].shape, 5, torch.bfloat16), True, -0.2, True, "negative scale")
+
+
+def test_bwd_bf16_full_size_sampled():
+    """The backward at the full prefill workload (B=8, L=4096, H_q=16, H_kv=8,
+    d=128, causal, 1% outlier keys), in the configuration the benchmark times:
+    dq and drho at 48 stratified query rows and dk, dv at 16 key rows among the
+    last 64 positions (the rows that see them are few), against the oracle's
+    row-by-row gradients, at the bf16 bar."""
+    shape = W.WORKLOADS["prefill_b8_l4096"]
+    x = W.make_prefill(shape, seed=40, device=DEV)
+    gen = torch.Generator(device=DEV).manual_seed(41)
+    dout = torch.randn(x["q"].shape, generator=gen, device=DEV).to(torch.bfloat16)
+    dq, drho, dk, dv = plx.prefill_bwd(x["q"], x["rho"], x["k"], x["v"], dout, causal=True,
+                                       softmax_scale=1.0)
+    torch.cuda.synchronize()
+    rows = W.sample_rows_prefill(shape, 48, seed=42)
+    rng = np.random.default_rng(43)
+    keys = np.stack([rng.integers(0, shape.B, 16), rng.integers(0, shape.Hkv, 16),
+                     rng.integers(shape.L - 64, shape.L, 16)], axis=1)
+    rq, rr, rk, rv = oracle.prefill_bwd_sampled(x["q"], x["rho"], x["k"], x["v"], dout, True,
+                                                1.0, rows, keys)
+    b, h, i = (torch.as_tensor(rows[:, c], device=DEV) for c in range(3))
+    kb, kh, kj = (torch.as_tensor(keys[:, c], device=DEV) for c in range(3))
+    check_out(to_np(dq[b, i, h]), rq, bf16=True, what="full-size dq")
+    check_out(to_np(drho[b, i, h]), rr, bf16=True, what="full-size drho")
+    check_out(to_np(dk[kb, kj, kh]), rk, bf16=True, what="full-size dk")
+    check_out(to_np(dv[kb, kj, kh]), rv, bf16=True, what="full-size dv")
