@@ -107,6 +107,15 @@ __device__ __forceinline__ uint64_t mnmajor_step(uint64_t desc, int kk) {
 }
 
 
+// The k-th unit of this CTA: rounds of gridDim.x units (heaviest first), in CTA
+// order in even rounds and in reverse in odd ones, so the heavy and light ends
+// of each round even out across the CTAs.  Past the last unit: -1.
+__device__ __forceinline__ int cta_unit(int k, int units) {
+  const long long g = gridDim.x;
+  const long long u = (long long)k * g + ((k & 1) ? g - 1 - blockIdx.x : (long long)blockIdx.x);
+  return u < units ? (int)u : -1;
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completing on an mbarrier
 // (addresses 16-byte aligned, size a multiple of 16 bytes).
 __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,
@@ -204,7 +213,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&vmap);
       int t = 0, ku = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+      for (int k = 0, u; ok && (u = cta_unit(k, p.units)) >= 0; ++k) {
         int b, h, mt, n;
         unit_of(u, b, h, mt, n);
         const int hk = h / p.G;
@@ -245,7 +254,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dg = smem_desc_sw128(smem_u32(sG), 16, 1024);
       int t = 0, ku = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+      for (int k = 0, u; ok && (u = cta_unit(k, p.units)) >= 0; ++k) {
         int b, h, mt, n;
         unit_of(u, b, h, mt, n);
         if (!mbar_wait(&bars->q_full, ku & 1, abort_flag, p.err)) break;
@@ -325,7 +334,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t my = (uint32_t)(half * 32);
     const float qs = p.qscale;
     int t = 0, ku = 0;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+    for (int k = 0, u; (u = cta_unit(k, p.units)) >= 0; ++k) {
       int b, h, mt, n;
       unit_of(u, b, h, mt, n);
       const int i = mt * kTileM + r;
@@ -534,7 +543,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&vmap);
       int t = 0, ku = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+      for (int k = 0, u; ok && (u = cta_unit(k, p.units)) >= 0; ++k) {
         int b, hk, kt, q0;
         unit_of(u, b, hk, kt, q0);
         if (ku > 0 && !mbar_wait(&bars->kv_empty, (ku - 1) & 1, abort_flag, p.err)) break;
@@ -581,7 +590,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dv = smem_desc_sw128(smem_u32(sV), 16, 1024);
       int t = 0, ku = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+      for (int k = 0, u; ok && (u = cta_unit(k, p.units)) >= 0; ++k) {
         int b, hk, kt, q0;
         unit_of(u, b, hk, kt, q0);
         if (!mbar_wait(&bars->kv_full, ku & 1, abort_flag, p.err)) break;
@@ -668,7 +677,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t my = (uint32_t)(half * 32);
     const float qs = p.qscale;
     int t = 0, ku = 0;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+    for (int k = 0, u; (u = cta_unit(k, p.units)) >= 0; ++k) {
       int b, hk, kt, q0;
       unit_of(u, b, hk, kt, q0);
       const int j = kt * kTileM + r;  // this thread's key
