@@ -44,18 +44,6 @@ __device__ __forceinline__ void load_slice<float>(const float* p, float (&f)[4],
     f[0] = w.x; f[1] = w.y; f[2] = f[3] = 0.f;
   }
 }
-template <>
-__device__ __forceinline__ void load_slice<__nv_bfloat16>(const __nv_bfloat16* p, float (&f)[4],
-                                                          int n) {
-  if (n == 4) {
-    const uint2 w = *reinterpret_cast<const uint2*>(p);
-    const float2 a = bf16x2_to_float2(w.x), b = bf16x2_to_float2(w.y);
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-  } else {
-    const float2 a = bf16x2_to_float2(*reinterpret_cast<const uint32_t*>(p));
-    f[0] = a.x; f[1] = a.y; f[2] = f[3] = 0.f;
-  }
-}
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
