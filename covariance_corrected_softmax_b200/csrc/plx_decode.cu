@@ -404,6 +404,14 @@ __global__ void __launch_bounds__(DecodeTile<T, D>::THREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  // Launched as a programmatic dependent of the previous kernel on the stream:
+  // this CTA may be resident before that kernel has finished (its launch and
+  // set-up overlap the other's tail), but it touches no global memory until
+  // that kernel has completed and its writes are visible.  The next kernel may
+  // likewise be scheduled as soon as SMs free up.
+  grid_dep_wait();
+  grid_dep_launch_dependents();
+
   if (tid == 0) {
     *abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
@@ -1071,7 +1079,19 @@ cudaError_t launch_decode_t(const DecodeMaps& m, const DecodeParams& p, cudaStre
                              : plx_decode_splitk_kernel<T, D, HPW, kDecContiguous>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<p.grid, Cfg::THREADS, smem, stream>>>(m.k, m.v, m.k_chunk, m.v_chunk, p);
+  // programmatic dependent launch: see the start of the kernel
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.grid);
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, m.k, m.v, m.k_chunk, m.v_chunk, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
