@@ -9,7 +9,8 @@ run on ``prefill_b8_l4096`` (B=8, L=4096, H_q=16, H_kv=8, d=128) and reported
 under ``"prefill"``, the long-context prefill ``prefill_b1_l32768`` (B=1,
 L=32768, H_q=32, H_kv=8) under ``"prefill_long"``, the gradients of the prefill
 (``plx_prefill_bwd`` on ``prefill_b8_l4096``, 16d flops per visible pair) under
-``"prefill_bwd"``, and the decode grid (batch
+``"prefill_bwd"``, the probe projection rho = x W_R^T at the prefill and the
+decode sizes under ``"probe_projection"``, and the decode grid (batch
 1-2048 x context 128-32768, ragged lengths) under ``"sweep"``: per cell the
 device time per call with L2 flushed before every call, HBM GB/s from the
 actual lengths and the fraction of the measured copy bandwidth.
@@ -422,6 +423,69 @@ def bench_prefill_bwd(plx, W, shape, steps, warmup, world, device, rank):
     return {"ms": ms, "clocks": clk.summary()}
 
 
+def bench_projection(plx, W, peaks, peak_src, device):
+    """The probe projection rho = x W_R^T (plx_probe_projection) at the prefill
+    workload's size (x [8 * 4096, 2048], W_R [16 * 128, 2048]; tensor-bound:
+    2 M N K flops, 20 calls alternating two inputs larger than L2) and at the
+    decode workload's (x [32, 2048]: bound by reading W_R, 8.4 MB; each call
+    timed alone after the L2 flush and clean-up read, median of 30)."""
+    import torch
+    res = {}
+    M, N, K = 8 * 4096, 16 * 128, 2048
+    xs = [W.make_probe_inputs((M,), K, N, seed=50 + c, device=device) for c in range(2)]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    for i in range(3):
+        plx.probe_projection(xs[i % 2][0], xs[i % 2][1], out=out)
+    torch.cuda.synchronize()
+    steps = 20
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_index()) as clk:
+        s.record()
+        for i in range(steps):
+            plx.probe_projection(xs[i % 2][0], xs[i % 2][1], out=out)
+        e.record()
+        torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    tflops = 2.0 * M * N * K / (ms / 1e3) / 1e12
+    res["prefill"] = {"M": M, "N": N, "K": K, "ms_per_call": ms, "tflops": tflops,
+                      "roofline": {"bound": "tensor", "achieved": tflops,
+                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                   "frac": tflops / peaks["bf16_tflops"],
+                                   "peak_source": f"{peak_src} bf16 dense (burst)"},
+                      "clocks": clk.summary()}
+    del xs, out
+    M = 32
+    x, w = W.make_probe_inputs((M,), K, N, seed=60, device=device)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    clean = torch.zeros(32 << 20, dtype=torch.int64, device=device)
+    for _ in range(3):
+        plx.probe_projection(x, w, out=out)
+    times = []
+    for _ in range(30):
+        flush.fill_(1)
+        clean.sum()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        plx.probe_projection(x, w, out=out)
+        e.record()
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e))
+    ms = statistics.median(times)
+    nbytes = 2.0 * (N * K + M * K + M * N)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    res["decode"] = {"M": M, "N": N, "K": K, "us_per_call": ms * 1e3, "gbs": gbs,
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                                  "peak_source": f"{peak_src} HBM copy bandwidth",
+                                  "bytes_per_call": nbytes},
+                     "launch_bound": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e6 < 20.0}
+    assert plx.device_error() == 0, "projection kernels reported a device error"
+    del x, w, out, flush, clean
+    torch.cuda.empty_cache()
+    return res
+
+
 def prefill_bwd_record(name, pshape, pr, psteps, peaks, peak_src):
     pms = pr["ms"] / psteps
     # 16d flops per visible (query, key) pair: the eight products S, T, GV,
@@ -658,6 +722,10 @@ def main():
         prefill_bwd = (prefill_bwd_record(PREFILL, pshape, pr, 10, peaks, peak_src)
                        if "ms" in pr else {"workload": PREFILL, **pr})
 
+    projection = None
+    if not args.no_prefill and world == 1:
+        projection = bench_projection(plx, W, peaks, peak_src, device)
+
     sweep = None
     if not args.no_sweep:
         with ClockSampler(gpu_index()) as clk:
@@ -695,6 +763,7 @@ def main():
         "prefill": prefill,
         "prefill_long": prefill_long,
         "prefill_bwd": prefill_bwd,
+        "probe_projection": projection,
         "sweep": sweep,
     }
     if rank == 0:
