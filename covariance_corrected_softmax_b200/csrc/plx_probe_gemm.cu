@@ -5,13 +5,31 @@
 //
 // For all tokens at once this is the GEMM rho[M, N] = x[M, K] W_R[N, K]^T
 // (M tokens, K = model width, N = H_q d), run on the 5th-generation tensor
-// cores for bf16: persistent CTAs over 128 x 128 output tiles (consecutive tiles
-// share the x tile, W_R stays in L2), a 6-stage ring of 128 x 64 x and W_R
-// tiles fed by TMA (128-byte swizzle), tcgen05.mma (M = 128, N = 128, K = 16)
-// issued by one thread into one of two TMEM accumulators, and four epilogue
-// warps that read the other accumulator (tcgen05.ld), round to bf16 and store
-// while the next tile accumulates.  fp32 inputs take a plain CUDA-core kernel
-// (the correctness path).
+// cores for bf16: a 192 KB ring fed by TMA (128-byte swizzle) with a 128 x 64
+// x tile and one or two W_R tiles per stage, tcgen05.mma (M = 128, N = 128,
+// K = 16) issued by one thread, and four epilogue warps that read a unit's
+// accumulators (tcgen05.ld) and round to bf16.  Products into the same
+// accumulator complete one after the other (each waits for the previous sum),
+// so every unit keeps two independent chains in flight: two adjacent N tiles
+// sharing the x tile (one accumulator each), or, for a single tile, the even
+// and odd k steps in two accumulators that the epilogue adds.  Two units in
+// flight (four accumulators, 512 columns): the epilogue of one overlaps the
+// products of the next.  Three schedules by the number of 128 x 128 output
+// tiles:
+//   * pairs of tiles (four ring stages), persistent CTAs, when their waves
+//     cost no more than single tiles' (a pair moves 1.5 times the bytes);
+//   * single tiles (six ring stages), persistent CTAs;
+//   * fewer tiles than half the SMs (the decode batch, M of a few dozen): a
+//     cluster of up to 8 CTAs per tile (the largest whose clusters all fit at
+//     once), each summing its share of the k blocks.  With so few tiles the
+//     time is the ring's round trips to memory, so spreading the W_R stream
+//     over more SMs is what shortens it.  The fp32 partial tiles meet in
+//     shared memory; every CTA of the cluster reads all of them (distributed
+//     shared memory) for its slice of the rows, adds them in rank order and
+//     stores.
+// fp32 inputs take a plain CUDA-core kernel (the correctness path).
+#include <atomic>
+
 #include "plx_launch.h"
 
 namespace plx {
@@ -19,14 +37,17 @@ namespace plx {
 namespace {
 
 constexpr int kPM = 128, kPN = 128, kPK = 64;  // output tile, k block (128-byte rows)
-constexpr int kPStages = 6;
+constexpr int kPRingBytes = 192 * 1024;       // four stages of pairs or six of single tiles
+constexpr int kPMaxStages = 6;
 constexpr int kPThreads = 256;                 // warps: 0 TMA, 1 MMA, 2 TMEM, 4-7 epilogue
 constexpr int kPTileBytes = kPM * kPK * 2;     // one A (or B) tile, 16 KB
-constexpr int kPStageBytes = 2 * kPTileBytes;
+constexpr int kPPartStride = kPN + 4;          // fp32 partial tile row (floats), conflict-free
 constexpr uint32_t kPIdesc = umma_idesc_f16kind(kPM, kPN, false, false);
+static_assert(kPM * kPPartStride * 4 <= kPRingBytes, "partial tile fits the ring");
+constexpr int kPMaxSplit = 8;  // cluster size (portable limit)
 
 struct ProjBars {
-  uint64_t full[kPStages], empty[kPStages];
+  uint64_t full[kPMaxStages], empty[kPMaxStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
 };
@@ -34,9 +55,47 @@ struct ProjBars {
 struct ProjParams {
   void* rho;
   int M, N, K;
-  int tiles_n, tiles, kblocks;
+  int tiles_n;   // 128-column output tiles
+  int pair;      // 1 or 2 N tiles per unit
+  int units_n;   // units per 128-row M tile
+  int units;
+  int kblocks;   // 64-wide k blocks
+  int ksplit;    // CTAs per unit (a cluster); 1: persistent CTAs
+  int stages;    // ring stages of stage_bytes: an x tile and `pair` W_R tiles
+  int stage_bytes;
   unsigned* err;
 };
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// every thread of every CTA of the cluster; shared-memory writes before it are
+// visible to the cluster's reads after it
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t local_addr, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_addr), "r"(rank));
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void unit_coords(const ProjParams& p, int u, int& mb, int& nb,
+                                            bool& two) {
+  mb = u / p.units_n;
+  nb = p.pair * (u % p.units_n);
+  two = p.pair == 2 && nb + 1 < p.tiles_n;
+}
 
 __global__ void __launch_bounds__(kPThreads, 1)
     plx_probe_gemm_kernel(const __grid_constant__ CUtensorMap xmap,
@@ -44,14 +103,25 @@ __global__ void __launch_bounds__(kPThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  ProjBars* bars = reinterpret_cast<ProjBars*>(smem + kPStages * kPStageBytes);
+  ProjBars* bars = reinterpret_cast<ProjBars*>(smem + kPRingBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // this CTA's units and k blocks: with ksplit > 1 the grid is one cluster
+  // of ksplit CTAs per unit, rank kr summing k blocks [kb0, kb1)
+  const int ks = p.ksplit;
+  const int kr = ks > 1 ? (int)cluster_rank() : 0;
+  const int kb0 = (int)((long long)p.kblocks * kr / ks);
+  const int kb1 = (int)((long long)p.kblocks * (kr + 1) / ks);
+  const int u_first = blockIdx.x / ks, u_step = gridDim.x / ks;
 
+  // a kernel launched after this one as its programmatic dependent (the
+  // attention that reads rho) waits for this grid's completion before it
+  // reads anything, so it may be placed on free SMs at once
+  grid_dep_launch_dependents();
   if (tid == 0) {
     *abort_flag = 0;
-    for (int s = 0; s < kPStages; ++s) {
+    for (int s = 0; s < p.stages; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
@@ -63,7 +133,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     fence_mbarrier_init();
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -76,21 +146,27 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&xmap);
       tma_prefetch_desc(&wmap);
-      long long it = 0;
+      int s = 0;            // ring stage
+      uint32_t round = 0;   // passes over the ring so far
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.tiles; u += gridDim.x) {
-        const int mb = u / p.tiles_n, nb = u % p.tiles_n;
-        for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-          const int s = (int)(it % kPStages);
-          if (it >= kPStages &&
-              !mbar_wait(&bars->empty[s], (uint32_t)(((it / kPStages) - 1) & 1), abort_flag, p.err)) {
+      for (int u = u_first; ok && u < p.units; u += u_step) {
+        int mb, nb;
+        bool two;
+        unit_coords(p, u, mb, nb, two);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (round > 0 && !mbar_wait(&bars->empty[s], (round - 1) & 1u, abort_flag, p.err)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + s * kPStageBytes;
-          mbar_arrive_expect_tx(&bars->full[s], kPStageBytes);
+          uint8_t* st = smem + s * p.stage_bytes;
+          mbar_arrive_expect_tx(&bars->full[s], (two ? 3 : 2) * kPTileBytes);
           tma_load_2d(st, &xmap, &bars->full[s], kb * kPK, mb * kPM);
           tma_load_2d(st + kPTileBytes, &wmap, &bars->full[s], kb * kPK, nb * kPN);
+          if (two) tma_load_2d(st + 2 * kPTileBytes, &wmap, &bars->full[s], kb * kPK, (nb + 1) * kPN);
+          if (++s == p.stages) {
+            s = 0;
+            ++round;
+          }
         }
       }
       if (*abort_flag) {
@@ -105,31 +181,50 @@ __global__ void __launch_bounds__(kPThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint64_t d0 = smem_desc_sw128(smem_u32(smem), 16, 1024);
-      long long it = 0;
+      int s = 0;
+      uint32_t round = 0;
       int lt = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.tiles; u += gridDim.x, ++lt) {
-        const int ab = lt & 1;
+      for (int u = u_first; ok && u < p.units; u += u_step, ++lt) {
+        const int ab = lt & 1;  // accumulators 2 ab and 2 ab + 1
+        int mb, nb;
+        bool two;
+        unit_coords(p, u, mb, nb, two);
         if (lt >= 2 &&
             !mbar_wait(&bars->acc_empty[ab], (uint32_t)(((lt >> 1) - 1) & 1), abort_flag, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-          const int s = (int)(it % kPStages);
-          if (!mbar_wait(&bars->full[s], (uint32_t)((it / kPStages) & 1), abort_flag, p.err)) {
+        const uint32_t acc0 = tbase + 2 * ab * kPN, acc1 = acc0 + kPN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&bars->full[s], round & 1u, abort_flag, p.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = (uint32_t)(s * kPStageBytes) >> 4;
-          const uint32_t sb = (uint32_t)(s * kPStageBytes + kPTileBytes) >> 4;
+          const uint32_t sa = (uint32_t)(s * p.stage_bytes) >> 4;
+          const uint32_t sb = (uint32_t)(s * p.stage_bytes + kPTileBytes) >> 4;
+          const uint32_t sc = (uint32_t)(s * p.stage_bytes + 2 * kPTileBytes) >> 4;
+          if (two) {
 #pragma unroll
-          for (int k = 0; k < kPK / 16; ++k)
-            umma_ss(tbase + ab * kPN, d0 + sa + 2 * k, d0 + sb + 2 * k, kPIdesc,
-                    (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < kPK / 16; ++k) {
+              const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+              umma_ss(acc0, d0 + sa + 2 * k, d0 + sb + 2 * k, kPIdesc, acc);
+              umma_ss(acc1, d0 + sa + 2 * k, d0 + sc + 2 * k, kPIdesc, acc);
+            }
+          } else {
+            // even k steps into acc0, odd ones into acc1
+#pragma unroll
+            for (int k = 0; k < kPK / 16; ++k)
+              umma_ss((k & 1) ? acc1 : acc0, d0 + sa + 2 * k, d0 + sb + 2 * k, kPIdesc,
+                      (kb > kb0 || k > 1) ? 1u : 0u);
+          }
           umma_commit(&bars->empty[s]);  // the stage is free once these MMAs complete
+          if (++s == p.stages) {
+            s = 0;
+            ++round;
+          }
         }
         if (!ok) break;
         umma_commit(&bars->acc_full[ab]);
@@ -146,17 +241,39 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int r = qd * 32 + lane;                // row of the tile = TMEM lane
     const uint32_t lane_addr = tbase + ((uint32_t)(qd * 32) << 16);
     int lt = 0;
-    for (int u = blockIdx.x; u < p.tiles; u += gridDim.x, ++lt) {
+    for (int u = u_first; u < p.units; u += u_step, ++lt) {
       const int ab = lt & 1;
       if (!mbar_wait(&bars->acc_full[ab], (uint32_t)((lt >> 1) & 1), abort_flag, p.err)) break;
       tc_fence_after();
-      const int mb = u / p.tiles_n, nb = u % p.tiles_n;
+      int mb, nb0;
+      bool two;
+      unit_coords(p, u, mb, nb0, two);
+      const uint32_t acc0 = lane_addr + 2 * ab * kPN;
       const long long row = (long long)mb * kPM + r;
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.rho) + row * p.N + (size_t)nb * kPN;
 #pragma unroll 1
-      for (int c = 0; c < kPN; c += 32) {
+      for (int c2 = 0; c2 < (two ? 2 : 1) * kPN; c2 += 32) {
         uint32_t v[32];
-        tmem_ld32_sync(lane_addr + ab * kPN + c, v);
+        tmem_ld32_sync(acc0 + c2, v);
+        if (!two) {
+          uint32_t w[32];
+          tmem_ld32_sync(acc0 + kPN + c2, w);
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w[j]));
+        }
+        if (ks > 1) {
+          // this CTA's share of the sum, kept in shared memory (the ring is idle:
+          // every load was consumed by the products that acc_full follows)
+          float* part = reinterpret_cast<float*>(smem) + r * kPPartStride + c2;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(part + 4 * q) =
+                make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                            __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+          continue;
+        }
+        const int nb = nb0 + c2 / kPN, c = c2 % kPN;
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.rho) + row * p.N + (size_t)nb * kPN;
         if (row < p.M) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -178,9 +295,50 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
   }
   __syncthreads();
+  if (ks > 1) {
+    // every CTA of the cluster reaches both barriers (all waits above are
+    // bounded); the second keeps each partial tile alive until all have read it
+    cluster_sync();
+    if (blockIdx.x / ks < p.units) {
+      int mb, nb;
+      bool two;
+      unit_coords(p, blockIdx.x / ks, mb, nb, two);
+      const int rows = min(kPM, p.M - mb * kPM);
+      const int items = rows * (kPN / 4);  // float4 groups of the tile
+      const int i0 = (int)((long long)items * kr / ks), i1 = (int)((long long)items * (kr + 1) / ks);
+      const uint32_t part0 = smem_u32(smem);
+      for (int i = i0 + tid; i < i1; i += kPThreads) {
+        const int row = i / (kPN / 4), c4 = i % (kPN / 4);
+        const uint32_t off = part0 + (uint32_t)(row * kPPartStride + 4 * c4) * 4u;
+        // all loads first (independent), then the sum in rank order
+        float4 b[kPMaxSplit];
+#pragma unroll
+        for (int s2 = 0; s2 < kPMaxSplit; ++s2)
+          if (s2 < ks) b[s2] = ld_cluster_f4(off, (uint32_t)s2);
+        float4 a = b[0];
+#pragma unroll
+        for (int s2 = 1; s2 < kPMaxSplit; ++s2)
+          if (s2 < ks) {
+            a.x += b[s2].x;
+            a.y += b[s2].y;
+            a.z += b[s2].z;
+            a.w += b[s2].w;
+          }
+        const int col = nb * kPN + 4 * c4;
+        if (col + 4 <= p.N) {
+          uint2 w;
+          w.x = float2_to_bf16x2(a.x, a.y);
+          w.y = float2_to_bf16x2(a.z, a.w);
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.rho) +
+                                    ((long long)mb * kPM + row) * p.N + col) = w;
+        }
+      }
+    }
+    cluster_sync();
+  }
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tbase, 256);
+    tmem_dealloc(tbase, 512);
   }
 }
 
@@ -218,6 +376,36 @@ cudaError_t encode_2d_sw128(CUtensorMap* map, const void* base, long long rows, 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// How many clusters of ks CTAs (smem bytes each) the device holds at once,
+// queried once per device and size; 0 if unknown.
+int max_active_clusters(int ks, int smem) {
+  static std::atomic<int> cache[16][kPMaxSplit + 1];  // 0: not queried, -1: none
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return 0;
+  std::atomic<int>& c = cache[dev][ks];
+  int n = c.load(std::memory_order_relaxed);
+  if (n == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)ks);
+    cfg.blockDim = dim3(kPThreads);
+    cfg.dynamicSmemBytes = smem;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, plx_probe_gemm_kernel, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    n = n > 0 ? n : -1;
+    c.store(n, std::memory_order_relaxed);
+  }
+  return n > 0 ? n : 0;
+}
+
 }  // namespace
 
 cudaError_t launch_probe_projection(const void* x, const void* w, void* rho, int M, int N, int K,
@@ -239,17 +427,56 @@ cudaError_t launch_probe_projection(const void* x, const void* w, void* rho, int
   p.M = M;
   p.N = N;
   p.K = K;
+  const long long mtiles = (M + kPM - 1) / kPM;
   p.tiles_n = (N + kPN - 1) / kPN;
-  const long long tiles = (long long)((M + kPM - 1) / kPM) * p.tiles_n;
-  if (tiles > 0x7fffffffll) return cudaErrorInvalidValue;
-  p.tiles = (int)tiles;
   p.kblocks = (K + kPK - 1) / kPK;
-  p.err = err;
-  const int smem = 1024 + kPStages * kPStageBytes + (int)sizeof(ProjBars) + 16;
+  const long long tiles = mtiles * p.tiles_n;
+  const int smem = 1024 + kPRingBytes + (int)sizeof(ProjBars) + 16;
   e = cudaFuncSetAttribute(plx_probe_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-  plx_probe_gemm_kernel<<<grid, kPThreads, smem, stream>>>(xm, wm, p);
+  p.pair = 1;
+  p.ksplit = 1;
+  // a pair of tiles moves 1.5 times a single tile's bytes through the ring:
+  // pairs when their waves cost no more than the single tiles' waves
+  const long long pairs = mtiles * ((p.tiles_n + 1) / 2);
+  if (3 * ((pairs + num_sms - 1) / num_sms) <= 2 * ((tiles + num_sms - 1) / num_sms) &&
+      pairs < tiles) {
+    p.pair = 2;
+  } else if (2 * tiles <= num_sms) {
+    // the largest cluster whose clusters all run at once (a second wave would
+    // cost more than the shorter k range saves)
+    for (int ks = kPMaxSplit; ks >= 2; --ks)
+      if (tiles * ks <= num_sms && ks <= p.kblocks && tiles <= max_active_clusters(ks, smem)) {
+        p.ksplit = ks;
+        break;
+      }
+  }
+  p.units_n = (p.tiles_n + p.pair - 1) / p.pair;
+  const long long units = mtiles * p.units_n;
+  if (units > 0x7fffffffll) return cudaErrorInvalidValue;
+  p.units = (int)units;
+  p.err = err;
+  p.stage_bytes = (1 + p.pair) * kPTileBytes;
+  p.stages = kPRingBytes / p.stage_bytes;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(kPThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  if (p.ksplit > 1) {
+    // one cluster per tile (units * ksplit <= num_sms here)
+    cfg.gridDim = dim3((unsigned)(units * p.ksplit));
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.ksplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  } else {
+    cfg.gridDim = dim3((unsigned)(units < num_sms ? units : num_sms));
+  }
+  e = cudaLaunchKernelEx(&cfg, plx_probe_gemm_kernel, xm, wm, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -36,9 +36,16 @@ def _check_projection(got, x, w, bf16):
     assert worst <= 1.0, f"projection error {worst:.3f} of its bound"
 
 
+# On 148 SMs the bf16 shapes reach each schedule: one tile (1x64x64,
+# 128x136x64), clusters of CTAs splitting K (5x256x72, 300x2048x2048,
+# 1000x384x520 with an uneven split, 32x2048x2048 the decode batch),
+# persistent single tiles (2000x1024x256) and pairs of tiles with an odd last
+# tile and ragged M, N, K (4100x1032x200).
 @pytest.mark.parametrize("M,N,K", [(1, 64, 64), (5, 256, 72), (128, 136, 64), (300, 2048, 2048),
-                                   (1000, 384, 520)],
-                         ids=["1x64x64", "5x256x72", "128x136x64", "300x2048x2048", "1000x384x520"])
+                                   (1000, 384, 520), (32, 2048, 2048), (2000, 1024, 256),
+                                   (4100, 1032, 200)],
+                         ids=["1x64x64", "5x256x72", "128x136x64", "300x2048x2048", "1000x384x520",
+                              "32x2048x2048", "2000x1024x256", "4100x1032x200"])
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
 def test_projection_matches_oracle(M, N, K, dt):
     x, w = W.make_probe_inputs((M,), K, N, seed=M + N + K, device=DEV, dtype=dt)
