@@ -6,16 +6,17 @@
 // For all tokens at once this is the GEMM rho[M, N] = x[M, K] W_R[N, K]^T
 // (M tokens, K = model width, N = H_q d), run on the 5th-generation tensor
 // cores for bf16: a 192 KB ring fed by TMA (128-byte swizzle) with a 128 x 64
-// x tile and one or two W_R tiles per stage, tcgen05.mma (M = 128, N = 128,
-// K = 16) issued by one thread, and four epilogue warps that read a unit's
-// accumulators (tcgen05.ld) and round to bf16.  Products into the same
+// x tile and one or two W_R tiles per stage, tcgen05.mma (M = 128, K = 16)
+// issued by one thread, and eight epilogue warps that read a unit's sums
+// (tcgen05.ld), round them to bf16 and store.  A unit is one 128 x 128 output
+// tile or a pair of adjacent ones; a pair's two W_R tiles lie back to back in
+// the stage, so one N = 256 product covers both.  Products into the same
 // accumulator complete one after the other (each waits for the previous sum),
-// so every unit keeps two independent chains in flight: two adjacent N tiles
-// sharing the x tile (one accumulator each), or, for a single tile, the even
-// and odd k steps in two accumulators that the epilogue adds.  Two units in
-// flight (four accumulators, 512 columns): the epilogue of one overlaps the
-// products of the next.  Three schedules by the number of 128 x 128 output
-// tiles:
+// and one such chain keeps the tensor core about half busy, so the even and
+// odd k steps accumulate into two accumulators (256 columns each) that the
+// epilogue adds: two chains in flight.  The epilogue releases TMEM as soon as
+// the sums are in registers and stores while the next unit accumulates.
+// Three schedules by the number of 128 x 128 output tiles:
 //   * pairs of tiles (four ring stages), persistent CTAs, when their waves
 //     cost no more than single tiles' (a pair moves 1.5 times the bytes);
 //   * single tiles (six ring stages), persistent CTAs;
@@ -39,16 +40,19 @@ namespace {
 constexpr int kPM = 128, kPN = 128, kPK = 64;  // output tile, k block (128-byte rows)
 constexpr int kPRingBytes = 192 * 1024;       // four stages of pairs or six of single tiles
 constexpr int kPMaxStages = 6;
-constexpr int kPThreads = 256;                 // warps: 0 TMA, 1 MMA, 2 TMEM, 4-7 epilogue
+constexpr int kPThreads = 384;                 // warps: 0 TMA, 1 MMA, 2 TMEM, 4-11 epilogue
+constexpr int kPEpiWarps = 8;                  // two per TMEM lane quadrant
+constexpr int kPAccCols = 256;                 // accumulator of the even k steps; the odd ones follow
 constexpr int kPTileBytes = kPM * kPK * 2;     // one A (or B) tile, 16 KB
 constexpr int kPPartStride = kPN + 4;          // fp32 partial tile row (floats), conflict-free
-constexpr uint32_t kPIdesc = umma_idesc_f16kind(kPM, kPN, false, false);
+constexpr uint32_t kPIdesc1 = umma_idesc_f16kind(kPM, kPN, false, false);      // one W_R tile
+constexpr uint32_t kPIdesc2 = umma_idesc_f16kind(kPM, 2 * kPN, false, false);  // two, as one N = 256 operand
 static_assert(kPM * kPPartStride * 4 <= kPRingBytes, "partial tile fits the ring");
 constexpr int kPMaxSplit = 8;  // cluster size (portable limit)
 
 struct ProjBars {
   uint64_t full[kPMaxStages], empty[kPMaxStages];
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t acc_full, acc_empty;
   uint64_t drain;
 };
 
@@ -125,10 +129,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&bars->acc_full[a], 1);
-      mbar_init(&bars->acc_empty[a], 4);  // one arrival per epilogue warp
-    }
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_empty, kPEpiWarps);  // one arrival per epilogue warp
     mbar_init(&bars->drain, 1);
     fence_mbarrier_init();
   }
@@ -186,17 +188,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
       int lt = 0;
       bool ok = true;
       for (int u = u_first; ok && u < p.units; u += u_step, ++lt) {
-        const int ab = lt & 1;  // accumulators 2 ab and 2 ab + 1
         int mb, nb;
         bool two;
         unit_coords(p, u, mb, nb, two);
-        if (lt >= 2 &&
-            !mbar_wait(&bars->acc_empty[ab], (uint32_t)(((lt >> 1) - 1) & 1), abort_flag, p.err)) {
+        // the epilogue has taken the previous unit's sums out of TMEM
+        if (lt > 0 && !mbar_wait(&bars->acc_empty, (uint32_t)((lt - 1) & 1), abort_flag, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t acc0 = tbase + 2 * ab * kPN, acc1 = acc0 + kPN;
+        // a pair's two W_R tiles are contiguous in the stage: one N = 256 operand
+        const uint32_t idesc = two ? kPIdesc2 : kPIdesc1;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&bars->full[s], round & 1u, abort_flag, p.err)) {
             ok = false;
@@ -205,21 +207,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
           tc_fence_after();
           const uint32_t sa = (uint32_t)(s * p.stage_bytes) >> 4;
           const uint32_t sb = (uint32_t)(s * p.stage_bytes + kPTileBytes) >> 4;
-          const uint32_t sc = (uint32_t)(s * p.stage_bytes + 2 * kPTileBytes) >> 4;
-          if (two) {
+          // even k steps into the first accumulator, odd ones into the second
 #pragma unroll
-            for (int k = 0; k < kPK / 16; ++k) {
-              const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
-              umma_ss(acc0, d0 + sa + 2 * k, d0 + sb + 2 * k, kPIdesc, acc);
-              umma_ss(acc1, d0 + sa + 2 * k, d0 + sc + 2 * k, kPIdesc, acc);
-            }
-          } else {
-            // even k steps into acc0, odd ones into acc1
-#pragma unroll
-            for (int k = 0; k < kPK / 16; ++k)
-              umma_ss((k & 1) ? acc1 : acc0, d0 + sa + 2 * k, d0 + sb + 2 * k, kPIdesc,
-                      (kb > kb0 || k > 1) ? 1u : 0u);
-          }
+          for (int k = 0; k < kPK / 16; ++k)
+            umma_ss(tbase + (k & 1) * kPAccCols, d0 + sa + 2 * k, d0 + sb + 2 * k, idesc,
+                    (kb > kb0 || k > 1) ? 1u : 0u);
           umma_commit(&bars->empty[s]);  // the stage is free once these MMAs complete
           if (++s == p.stages) {
             s = 0;
@@ -227,7 +219,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           }
         }
         if (!ok) break;
-        umma_commit(&bars->acc_full[ab]);
+        umma_commit(&bars->acc_full);
       }
       // every MMA must have completed before the columns are released
       umma_commit(&bars->drain);
@@ -237,61 +229,60 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
-    const int qd = warp & 3;                     // TMEM lane quadrant
+    const int qd = warp & 3;                     // TMEM lane quadrant (warp id mod 4)
+    const int half = (warp - 4) >> 2;            // which half of the unit's columns
     const int r = qd * 32 + lane;                // row of the tile = TMEM lane
     const uint32_t lane_addr = tbase + ((uint32_t)(qd * 32) << 16);
     int lt = 0;
     for (int u = u_first; u < p.units; u += u_step, ++lt) {
-      const int ab = lt & 1;
-      if (!mbar_wait(&bars->acc_full[ab], (uint32_t)((lt >> 1) & 1), abort_flag, p.err)) break;
+      if (!mbar_wait(&bars->acc_full, (uint32_t)(lt & 1), abort_flag, p.err)) break;
       tc_fence_after();
       int mb, nb0;
       bool two;
       unit_coords(p, u, mb, nb0, two);
-      const uint32_t acc0 = lane_addr + 2 * ab * kPN;
-      const long long row = (long long)mb * kPM + r;
-#pragma unroll 1
-      for (int c2 = 0; c2 < (two ? 2 : 1) * kPN; c2 += 32) {
-        uint32_t v[32];
-        tmem_ld32_sync(acc0 + c2, v);
-        if (!two) {
-          uint32_t w[32];
-          tmem_ld32_sync(acc0 + kPN + c2, w);
+      const int hcols = two ? kPN : kPN / 2;     // this warp's columns
+      const int c0 = half * hcols;               // the first, within the unit
+      uint32_t packed[kPN / 2];                  // bf16 pairs of the sums
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w[j]));
-        }
-        if (ks > 1) {
-          // this CTA's share of the sum, kept in shared memory (the ring is idle:
-          // every load was consumed by the products that acc_full follows)
-          float* part = reinterpret_cast<float*>(smem) + r * kPPartStride + c2;
+      for (int j = 0; j < kPN / 32; ++j) {
+        if (32 * j < hcols) {
+          uint32_t a[32], b[32];
+          tmem_ld2x32_sync(lane_addr + c0 + 32 * j, lane_addr + kPAccCols + c0 + 32 * j, a, b);
+          if (ks > 1) {
+            // this CTA's share of the sum, kept in shared memory (the ring is
+            // idle: every load was consumed by the products acc_full follows)
+            float* part = reinterpret_cast<float*>(smem) + r * kPPartStride + c0 + 32 * j;
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(part + 4 * q) =
-                make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                            __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-          continue;
-        }
-        const int nb = nb0 + c2 / kPN, c = c2 % kPN;
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.rho) + row * p.N + (size_t)nb * kPN;
-        if (row < p.M) {
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<float4*>(part + 4 * q) = make_float4(
+                  __uint_as_float(a[4 * q]) + __uint_as_float(b[4 * q]),
+                  __uint_as_float(a[4 * q + 1]) + __uint_as_float(b[4 * q + 1]),
+                  __uint_as_float(a[4 * q + 2]) + __uint_as_float(b[4 * q + 2]),
+                  __uint_as_float(a[4 * q + 3]) + __uint_as_float(b[4 * q + 3]));
+          } else {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = nb * kPN + c + 8 * q;
-            if (col + 8 <= p.N) {
-              uint4 w;
-              w.x = float2_to_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1]));
-              w.y = float2_to_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-              w.z = float2_to_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-              w.w = float2_to_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-              *reinterpret_cast<uint4*>(dst + c + 8 * q) = w;
-            }
+            for (int q = 0; q < 16; ++q)
+              packed[16 * j + q] =
+                  float2_to_bf16x2(__uint_as_float(a[2 * q]) + __uint_as_float(b[2 * q]),
+                                   __uint_as_float(a[2 * q + 1]) + __uint_as_float(b[2 * q + 1]));
           }
         }
       }
+      // the sums are in registers: the next unit may overwrite the accumulators
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);
+      if (lane == 0) mbar_arrive(&bars->acc_empty);
+      const long long row = (long long)mb * kPM + r;
+      if (ks == 1 && row < p.M) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.rho) + row * p.N;
+#pragma unroll
+        for (int g = 0; g < kPN / 8; ++g) {
+          const int col = nb0 * kPN + c0 + 8 * g;
+          if (8 * g < hcols && col + 8 <= p.N)
+            *reinterpret_cast<uint4*>(dst + col) =
+                make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+        }
+      }
     }
   }
   __syncthreads();
