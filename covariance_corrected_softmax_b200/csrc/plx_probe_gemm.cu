@@ -333,6 +333,232 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Pairs of SMs (tcgen05 cta_group::2): for many tiles, a cluster of two CTAs
+// computes a 256 x 256 output tile with M = 256, N = 256 products issued by
+// the even CTA.  Each CTA stages its own 128 rows of x and its own 128 rows of
+// W_R (one tile each, 32 KB per k block, six stages), and each SM's tensor
+// core multiplies its x rows by both CTAs' W_R rows, so a CTA moves 32 KB
+// through shared memory per k block for a 128 x 256 share of the output where
+// the one-SM pair of tiles moves 48 KB.  Both CTAs' loads complete on the even
+// CTA's stage barrier, the products' completion is signalled to both CTAs'
+// barriers, and both CTAs' epilogue warps release the accumulators on the even
+// CTA's barrier.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kPIdescPair = umma_idesc_f16kind(2 * kPM, 2 * kPN, false, false);
+constexpr int kPPairStages = kPRingBytes / (2 * kPTileBytes);
+static_assert(kPPairStages <= kPMaxStages, "stage barriers");
+
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local_addr, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_addr), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(smem_dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on the barrier at this offset in each CTA of `mask` once the products
+// issued so far have completed
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+// a tile into this CTA's shared memory, completing on a barrier of either CTA
+// of the pair (bar: shared::cluster address)
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// p.units = ceil(M / 256) ceil(N / 256) (units_n per 256-row M tile); the
+// grid is two CTAs (one cluster) per resident unit.
+__global__ void __launch_bounds__(kPThreads, 1)
+    plx_probe_gemm_pair_kernel(const __grid_constant__ CUtensorMap xmap,
+                               const __grid_constant__ CUtensorMap wmap, const ProjParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  ProjBars* bars = reinterpret_cast<ProjBars*>(smem + kPRingBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();  // 0: issues the products
+  const int u_first = blockIdx.x / 2, u_step = gridDim.x / 2;
+  constexpr int kStageBytes = 2 * kPTileBytes;  // x rows and W_R rows of this CTA
+
+  grid_dep_launch_dependents();
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kPPairStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_empty, 2 * kPEpiWarps);  // both CTAs' epilogue warps
+    mbar_init(&bars->drain, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM of both allocated
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      tma_prefetch_desc(&xmap);
+      tma_prefetch_desc(&wmap);
+      const uint32_t full0 = cluster_addr(smem_u32(&bars->full[0]), 0);
+      int s = 0;
+      uint32_t round = 0;
+      bool ok = true;
+      for (int u = u_first; ok && u < p.units; u += u_step) {
+        const int xrow = (u / p.units_n) * 2 * kPM + (int)rank * kPM;
+        const int wrow = (u % p.units_n) * 2 * kPN + (int)rank * kPN;
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (round > 0 && !mbar_wait(&bars->empty[s], (round - 1) & 1u, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kStageBytes;
+          if (rank == 0) mbar_arrive_expect_tx(&bars->full[s], 2 * kStageBytes);
+          tma_load_2d_pair(st, &xmap, full0 + 8u * (uint32_t)s, kb * kPK, xrow);
+          tma_load_2d_pair(st + kPTileBytes, &wmap, full0 + 8u * (uint32_t)s, kb * kPK, wrow);
+          if (++s == kPPairStages) {
+            s = 0;
+            ++round;
+          }
+        }
+      }
+      if (*abort_flag) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 100000) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      const uint64_t d0 = smem_desc_sw128(smem_u32(smem), 16, 1024);
+      int s = 0;
+      uint32_t round = 0;
+      int lt = 0;
+      bool ok = true;
+      for (int u = u_first; ok && u < p.units; u += u_step, ++lt) {
+        if (lt > 0 && !mbar_wait(&bars->acc_empty, (uint32_t)((lt - 1) & 1), abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(&bars->full[s], round & 1u, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = (uint32_t)(s * kStageBytes) >> 4;
+          const uint32_t sb = (uint32_t)(s * kStageBytes + kPTileBytes) >> 4;
+#pragma unroll
+          for (int k = 0; k < kPK / 16; ++k)
+            umma_ss_pair(tbase + (k & 1) * kPAccCols, d0 + sa + 2 * k, d0 + sb + 2 * k,
+                         kPIdescPair, (kb > 0 || k > 1) ? 1u : 0u);
+          umma_commit_pair(&bars->empty[s], 0x3);  // both CTAs' stage s is free
+          if (++s == kPPairStages) {
+            s = 0;
+            ++round;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&bars->acc_full, 0x3);
+      }
+      umma_commit_pair(&bars->drain, 0x1);
+      volatile int never = 0;
+      mbar_wait(&bars->drain, 0, &never, p.err);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int qd = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int r = qd * 32 + lane;
+    const uint32_t lane_addr = tbase + ((uint32_t)(qd * 32) << 16);
+    const uint32_t acc_empty0 = cluster_addr(smem_u32(&bars->acc_empty), 0);
+    int lt = 0;
+    for (int u = u_first; u < p.units; u += u_step, ++lt) {
+      if (!mbar_wait(&bars->acc_full, (uint32_t)(lt & 1), abort_flag, p.err)) break;
+      tc_fence_after();
+      const int c0 = half * kPN;  // this warp's 128 of the tile's 256 columns
+      uint32_t packed[kPN / 2];
+#pragma unroll
+      for (int j = 0; j < kPN / 16; ++j) {
+        uint32_t a[16], b[16];
+        tmem_ld2x16_sync(lane_addr + c0 + 16 * j, lane_addr + kPAccCols + c0 + 16 * j, a, b);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          packed[8 * j + q] =
+              float2_to_bf16x2(__uint_as_float(a[2 * q]) + __uint_as_float(b[2 * q]),
+                               __uint_as_float(a[2 * q + 1]) + __uint_as_float(b[2 * q + 1]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0);
+      const long long row = (long long)(u / p.units_n) * 2 * kPM + (long long)rank * kPM + r;
+      if (row < p.M) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.rho) + row * p.N;
+#pragma unroll
+        for (int g = 0; g < kPN / 8; ++g) {
+          const int col = (u % p.units_n) * 2 * kPN + c0 + 8 * g;
+          if (col + 8 <= p.N)
+            *reinterpret_cast<uint4*>(dst + col) =
+                make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // no product, load or remote arrival of either CTA is still pending
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tbase, 512);
+  }
+}
+
 // fp32: one thread per output, 16 x 16 output tiles through shared memory.
 __global__ void __launch_bounds__(256)
     plx_probe_simt_kernel(const float* x, const float* w, float* rho, int M, int N, int K) {
@@ -367,13 +593,14 @@ cudaError_t encode_2d_sw128(CUtensorMap* map, const void* base, long long rows, 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// How many clusters of ks CTAs (smem bytes each) the device holds at once,
-// queried once per device and size; 0 if unknown.
-int max_active_clusters(int ks, int smem) {
-  static std::atomic<int> cache[16][kPMaxSplit + 1];  // 0: not queried, -1: none
+// How many clusters of ks CTAs (smem bytes each) of the kernel (0: the one-SM
+// kernel, 1: the SM-pair kernel) the device holds at once, queried once per
+// device, kernel and size; 0 if unknown.
+int max_active_clusters(int kernel, int ks, int smem) {
+  static std::atomic<int> cache[16][2][kPMaxSplit + 1];  // 0: not queried, -1: none
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return 0;
-  std::atomic<int>& c = cache[dev][ks];
+  std::atomic<int>& c = cache[dev][kernel][ks];
   int n = c.load(std::memory_order_relaxed);
   if (n == 0) {
     cudaLaunchConfig_t cfg = {};
@@ -387,7 +614,9 @@ int max_active_clusters(int ks, int smem) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, plx_probe_gemm_kernel, &cfg) != cudaSuccess) {
+    const cudaError_t e = kernel ? cudaOccupancyMaxActiveClusters(&n, plx_probe_gemm_pair_kernel, &cfg)
+                                 : cudaOccupancyMaxActiveClusters(&n, plx_probe_gemm_kernel, &cfg);
+    if (e != cudaSuccess) {
       (void)cudaGetLastError();
       n = 0;
     }
@@ -423,6 +652,37 @@ cudaError_t launch_probe_projection(const void* x, const void* w, void* rho, int
   p.kblocks = (K + kPK - 1) / kPK;
   const long long tiles = mtiles * p.tiles_n;
   const int smem = 1024 + kPRingBytes + (int)sizeof(ProjBars) + 16;
+  p.err = err;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(kPThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  // SM pairs when every pair has a 256 x 256 tile to work on
+  const long long units2 = ((M + 2 * kPM - 1) / (2 * kPM)) * ((N + 2 * kPN - 1) / (2 * kPN));
+  if (units2 >= num_sms / 2 && units2 <= 0x7fffffffll) {
+    e = cudaFuncSetAttribute(plx_probe_gemm_pair_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int pairs = max_active_clusters(1, 2, smem);
+    if (pairs > 0) {
+      p.units = (int)units2;
+      p.units_n = (N + 2 * kPN - 1) / (2 * kPN);
+      p.pair = 2;
+      p.ksplit = 2;
+      p.stage_bytes = 2 * kPTileBytes;
+      p.stages = kPPairStages;
+      const long long clusters = units2 < pairs ? units2 : pairs;
+      cfg.gridDim = dim3((unsigned)(2 * clusters));
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      return cudaLaunchKernelEx(&cfg, plx_probe_gemm_pair_kernel, xm, wm, p);
+    }
+  }
   e = cudaFuncSetAttribute(plx_probe_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   p.pair = 1;
@@ -437,7 +697,7 @@ cudaError_t launch_probe_projection(const void* x, const void* w, void* rho, int
     // the largest cluster whose clusters all run at once (a second wave would
     // cost more than the shorter k range saves)
     for (int ks = kPMaxSplit; ks >= 2; --ks)
-      if (tiles * ks <= num_sms && ks <= p.kblocks && tiles <= max_active_clusters(ks, smem)) {
+      if (tiles * ks <= num_sms && ks <= p.kblocks && tiles <= max_active_clusters(0, ks, smem)) {
         p.ksplit = ks;
         break;
       }
@@ -446,14 +706,8 @@ cudaError_t launch_probe_projection(const void* x, const void* w, void* rho, int
   const long long units = mtiles * p.units_n;
   if (units > 0x7fffffffll) return cudaErrorInvalidValue;
   p.units = (int)units;
-  p.err = err;
   p.stage_bytes = (1 + p.pair) * kPTileBytes;
   p.stages = kPRingBytes / p.stage_bytes;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.blockDim = dim3(kPThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
   if (p.ksplit > 1) {
     // one cluster per tile (units * ksplit <= num_sms here)
     cfg.gridDim = dim3((unsigned)(units * p.ksplit));
