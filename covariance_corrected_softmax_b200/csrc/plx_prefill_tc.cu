@@ -10,8 +10,8 @@
 // which is o_SA - Sigma_KV^T rho written so that one pass over the keys and
 // values feeds both branches (page 3: the KV stream is reused by both).
 //
-// Per CTA (persistent; one 128-row query tile per work unit, heaviest causal
-// tiles first):
+// Per CTA (persistent; one 128-row query tile per work unit, bands of the
+// heaviest causal tiles first, a band's units grouped by KV head):
 //   warp 0      TMA producer: Q and R tiles once per unit, K and V tiles of 64
 //               keys into a 4-stage ring (128-byte swizzled, UMMA-canonical).
 //   warp 1      S/T issuer (one thread): S = Q K^T and T = R K^T of each key
@@ -178,6 +178,7 @@ struct Unit {
 
 template <bool VARLEN>
 __device__ __forceinline__ Unit unit_of(const TcParams& p, int u);
+constexpr int kBand = 8;  // query tiles per band of the fixed-shape unit order
 
 // The units the recomputing instance (SAFE) takes: a bit per unit of this CTA
 // (u = blockIdx.x + k gridDim.x), set where the fast instance left the marker.
@@ -210,10 +211,29 @@ template <bool VARLEN>
 __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
   Unit x;
   const int bh = p.B * p.Hq;
-  x.mt = p.nqt - 1 - u / bh;  // heaviest (last) query tiles first
-  const int r = u % bh;
-  x.b = r / p.Hq;
-  x.h = r % p.Hq;
+  if constexpr (VARLEN) {
+    x.mt = p.nqt - 1 - u / bh;  // heaviest (last) query tiles first
+    const int r = u % bh;
+    x.b = r / p.Hq;
+    x.h = r % p.Hq;
+  } else {
+    // Bands of kBand query tiles, the heaviest (last) band first, which keeps
+    // the causal work balanced over the persistent CTAs; within a band the
+    // units of one (batch, KV head) are consecutive (the group's query heads
+    // side by side), so the CTAs running at one time share a few K/V streams
+    // and read them from L2 rather than all B H_kv of them.  The tiles of a
+    // group run heaviest first in even groups and lightest first in odd ones,
+    // which evens out the work of the CTAs that take every gridDim-th unit.
+    const int band = u / (kBand * bh);
+    const int top = p.nqt - band * kBand;  // one past the band's heaviest tile
+    const int w = min(kBand, top);         // query tiles in the band
+    const int r = u - band * kBand * bh;
+    const int grp = r / (w * p.G), i = r % (w * p.G);
+    const int k = (grp & 1) ? w - 1 - i / p.G : i / p.G;
+    x.b = grp / p.Hkv;
+    x.h = (grp % p.Hkv) * p.G + i % p.G;
+    x.mt = top - 1 - k;
+  }
   x.bad = false;
   if constexpr (VARLEN) {
     const int s0 = p.cu_seqlens[x.b], s1 = p.cu_seqlens[x.b + 1];
