@@ -497,16 +497,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
+          // S and T products alternate, so that the two accumulate chains
+          // are in flight together
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = ((k >> 2) * C::Q_BOX + (k & 3) * 32) >> 4;
             const uint32_t koff = (C::k_box(st, k >> 2) + (k & 3) * 32) >> 4;
             umma_ss(tbase + C::COL_S, dq + off, dkv + koff, C::IDESC_ST, k > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = ((k >> 2) * C::Q_BOX + (k & 3) * 32) >> 4;
-            const uint32_t koff = (C::k_box(st, k >> 2) + (k & 3) * 32) >> 4;
             umma_ss(tbase + C::COL_T, dr + off, dkv + koff, C::IDESC_ST, k > 0 ? 1u : 0u);
           }
           umma_commit(&bars->s_full);
@@ -562,15 +559,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int s = 1; s < kStages; ++s)
             if (st == s) bv = dv[s];
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
+          for (int kk = 0; kk < kBN / 16; ++kk) {
             umma_ts(tbase + C::COL_O, tbase + C::COL_P + 8 * kk,
                     bv + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
                     (j == 0 && kk == 0) ? 0u : 1u);
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
             umma_ts(tbase + C::COL_U, tbase + C::COL_PT + 8 * kk,
                     bv + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV,
                     (j == 0 && kk == 0) ? 0u : 1u);
+          }
           umma_commit(&bars->o_done);
           umma_commit(&bars->kv_empty[st]);
         }
