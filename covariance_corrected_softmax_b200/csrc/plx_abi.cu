@@ -179,6 +179,7 @@ plx_status prefill_impl(const void* q, const void* rho, const void* k, const voi
                         bool check_only);
 
 // rho[M, N] = x[M, K] w_r[N, K]^T (all checks first; check_only stops there).
+constexpr int kMaxProjRows = 0x7FFFFE00;  // 2^31 - 512
 plx_status projection_impl(const void* x, const void* w_r, void* rho, int M, int N, int K,
                            plx_dtype dtype, void* stream, bool check_only) {
   t_last_cuda_error = 0;
@@ -188,6 +189,10 @@ plx_status projection_impl(const void* x, const void* w_r, void* rho, int M, int
   if (!x || !w_r || !rho || !aligned16(x) || !aligned16(w_r) || !aligned16(rho))
     return PLX_ERR_INVALID_ARGUMENT;
   if (dtype == PLX_BF16 && (K % 8 != 0 || N % 8 != 0)) return PLX_ERR_UNSUPPORTED;
+  // tile row coordinates (up to 255 past M or N) are 32-bit; the fp32
+  // kernel's grid holds 65535 tiles of 16 columns
+  if (dtype == PLX_BF16 && (M > kMaxProjRows || N > kMaxProjRows)) return PLX_ERR_UNSUPPORTED;
+  if (dtype == PLX_F32 && N > 65535 * 16) return PLX_ERR_UNSUPPORTED;
   if (check_only) return PLX_OK;
   int sms = 0;
   unsigned* err = nullptr;

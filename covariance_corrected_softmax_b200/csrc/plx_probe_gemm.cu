@@ -559,16 +559,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
-// fp32: one thread per output, 16 x 16 output tiles through shared memory.
+// fp32: one thread per output, 16 x 16 output tiles through shared memory
+// (blockIdx.x over the rows, so M is limited only by the grid's x extent).
 __global__ void __launch_bounds__(256)
     plx_probe_simt_kernel(const float* x, const float* w, float* rho, int M, int N, int K) {
   __shared__ float xs[16][17], ws[16][17];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const long long m = (long long)blockIdx.y * 16 + ty;
-  const long long n = (long long)blockIdx.x * 16 + tx;
+  const long long m = (long long)blockIdx.x * 16 + ty;
+  const long long n = (long long)blockIdx.y * 16 + tx;
   float acc = 0.f;
   for (int k0 = 0; k0 < K; k0 += 16) {
-    const long long mx = (long long)blockIdx.y * 16 + ty, nw = (long long)blockIdx.x * 16 + ty;
+    const long long mx = (long long)blockIdx.x * 16 + ty, nw = (long long)blockIdx.y * 16 + ty;
     xs[ty][tx] = (mx < M && k0 + tx < K) ? x[mx * K + k0 + tx] : 0.f;
     ws[ty][tx] = (nw < N && k0 + tx < K) ? w[nw * K + k0 + tx] : 0.f;
     __syncthreads();
@@ -632,7 +633,7 @@ cudaError_t launch_probe_projection(const void* x, const void* w, void* rho, int
                                     bool bf16, int num_sms, unsigned* err, cudaStream_t stream) {
   if (M == 0 || N == 0) return cudaSuccess;
   if (!bf16) {
-    dim3 grid((N + 15) / 16, (M + 15) / 16);
+    dim3 grid((M + 15) / 16, (N + 15) / 16);
     plx_probe_simt_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(x),
                                                     static_cast<const float*>(w),
                                                     static_cast<float*>(rho), M, N, K);

@@ -149,9 +149,9 @@ PLX_API plx_status plx_prefill_varlen(const void* q, const void* rho, const void
  *   w_r  : [N, K]  W_R, row n = output feature n (N = H_q * d for the
  *                  attention's probe layout [.., H_q, d])
  *   rho  : [M, N]  written, in dtype
- * PLX_BF16 runs on the tensor cores and needs K % 8 == 0 and N % 8 == 0
- * (else PLX_ERR_UNSUPPORTED); PLX_F32 on the CUDA cores.  M == 0 or N == 0 is
- * a no-op; K >= 1.
+ * PLX_BF16 runs on the tensor cores and needs K % 8 == 0, N % 8 == 0 and
+ * M, N <= 2^31 - 512; PLX_F32 runs on the CUDA cores and needs N <= 1048560
+ * (else PLX_ERR_UNSUPPORTED).  M == 0 or N == 0 is a no-op; K >= 1.
  */
 PLX_API plx_status plx_probe_projection(const void* x, const void* w_r, void* rho, int M, int N,
                                         int K, plx_dtype dtype, void* stream);

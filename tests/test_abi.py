@@ -244,6 +244,10 @@ def test_probe_projection_rejects():
     assert f(FAKE, FAKE + 8, FAKE, 4, 16, 8, plx.PLX_BF16, None) == INV
     assert f(FAKE, FAKE, FAKE, 4, 16, 12, plx.PLX_BF16, None) == plx.PLX_ERR_UNSUPPORTED  # K % 8
     assert f(FAKE, FAKE, FAKE, 4, 20, 8, plx.PLX_BF16, None) == plx.PLX_ERR_UNSUPPORTED  # N % 8
+    big = 2 ** 31 - 504  # tile row coordinates would pass 2^31
+    assert f(FAKE, FAKE, FAKE, big, 16, 8, plx.PLX_BF16, None) == plx.PLX_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 4, big, 8, plx.PLX_BF16, None) == plx.PLX_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 4, 65535 * 16 + 1, 8, plx.PLX_F32, None) == plx.PLX_ERR_UNSUPPORTED
     assert f(None, None, None, 0, 16, 8, plx.PLX_BF16, None) == plx.PLX_OK  # M = 0: no-op
 
 
