@@ -16,9 +16,12 @@
 // odd k steps accumulate into two accumulators (256 columns each) that the
 // epilogue adds: two chains in flight.  The epilogue releases TMEM as soon as
 // the sums are in registers and stores while the next unit accumulates.
-// Three schedules by the number of 128 x 128 output tiles:
-//   * pairs of tiles (four ring stages), persistent CTAs, when their waves
-//     cost no more than single tiles' (a pair moves 1.5 times the bytes);
+// Four schedules by the number of output tiles:
+//   * at least one 256 x 256 tile per pair of SMs: the SM-pair kernel below
+//     (tcgen05 cta_group::2), persistent clusters of two CTAs;
+//   * pairs of 128 x 128 tiles (four ring stages), persistent CTAs, when
+//     their waves cost no more than single tiles' (a pair moves 1.5 times the
+//     bytes);
 //   * single tiles (six ring stages), persistent CTAs;
 //   * fewer tiles than half the SMs (the decode batch, M of a few dozen): a
 //     cluster of up to 8 CTAs per tile (the largest whose clusters all fit at
