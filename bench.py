@@ -132,17 +132,20 @@ def barrier(world: int):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while it runs."""
+    """nvidia-smi clocks and throttle reasons, sampled every 20 ms around the
+    timed region; the summary keeps the samples taken inside it (host clock
+    between entering and leaving the `with` block, 0.3 s pre-roll excluded)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int, period_ms: int = 50):
+    def __init__(self, gpu_index: int, period_ms: int = 20):
         self.idx = gpu_index
         self.period = period_ms
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -155,9 +158,11 @@ class ClockSampler:
             time.sleep(0.3)
         except OSError:
             self.proc = None
+        self.t0 = time.time()
         return self
 
     def __exit__(self, *exc):
+        self.t1 = time.time()
         if self.proc is not None:
             time.sleep(0.1)
             self.proc.terminate()
@@ -166,25 +171,44 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
+    @staticmethod
+    def _epoch(stamp):
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(stamp, fmt).timestamp()
+            except ValueError:
+                continue
+        return None
+
     def summary(self):
         rows = []
         if self.path and os.path.exists(self.path):
             with open(self.path) as f:
                 for line in f:
                     p = [x.strip() for x in line.split(",")]
-                    if len(p) < 9:
+                    if len(p) < 10:
                         continue
                     try:
-                        rows.append((float(p[1]), float(p[2]), float(p[3]), p[5:9]))
+                        rows.append((self._epoch(p[0]), float(p[2]), float(p[3]), float(p[4]),
+                                     p[6:10]))
                     except ValueError:
                         continue
             os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        window = [r for r in rows if r[0] is not None and self.t0 is not None and
+                  self.t0 <= r[0] <= self.t1 + self.period / 1000.0]
+        if not window:
+            # a region shorter than the sampling period: the first sample after it began
+            after = [r for r in rows if r[0] is not None and self.t0 is not None and r[0] >= self.t0]
+            window = after[:1] or rows[-1:]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "power_w_max": max(r[2] for r in rows), "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for r in window for i, v in enumerate(r[4]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in window),
+                "sm_max_mhz": max(r[2] for r in rows),
+                "power_w_max": max(r[3] for r in window), "reasons": reasons,
+                "samples": len(window),
+                "window_ms": round(1000.0 * (self.t1 - self.t0), 1) if self.t1 else None}
 
 
 # ------------------------------------------------------------------------ decode

@@ -1,4 +1,5 @@
-"""Host logic of bench.py for more than one rank, on CPU with the gloo backend.
+"""Host logic of bench.py, on CPU: the paths for more than one rank (gloo
+backend) and the clock record.
 
 The GPU runs of this build have one GPU, so the N > 1 paths of the benchmark
 (max-over-ranks timing, barriers, the whole-job rate, the reference arm's
@@ -8,6 +9,7 @@ import datetime
 import os
 import socket
 import sys
+import tempfile
 
 import pytest
 
@@ -103,3 +105,28 @@ def test_recorded_traffic_follows_the_source_digest(tmp_path, monkeypatch):
     assert bench.recorded_traffic("k1", "other", ["a.cu"]) is None
     (csrc / "a.cu").write_text("kernel v2\n")  # the kernel changed since the capture
     assert bench.recorded_traffic("k1", "w1", ["a.cu"]) is None
+
+
+def test_clock_summary_keeps_the_timed_window():
+    """The clock record is the median of the samples taken inside the timed
+    region: pre-roll and tail samples at idle clocks are left out."""
+    clk = bench.ClockSampler(0)
+    t0 = datetime.datetime(2026, 1, 2, 3, 4, 5).timestamp()
+
+    def row(dt, mhz, power, cap):
+        stamp = datetime.datetime.fromtimestamp(t0 + dt).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return (f"{stamp}, 0, {mhz}, 1965, {power}, 0x0, Not Active, Not Active, Not Active, "
+                f"{'Active' if cap else 'Not Active'}\n")
+
+    fd, clk.path = tempfile.mkstemp(suffix=".csv")
+    with os.fdopen(fd, "w") as f:
+        for k in range(15):  # pre-roll at idle
+            f.write(row(-0.3 + 0.02 * k, 1965, 100.0, False))
+        for k in range(5):  # the timed region, under the power cap
+            f.write(row(0.005 + 0.02 * k, 1700 + k, 900.0, True))
+        f.write(row(0.3, 1965, 120.0, False))  # tail
+    clk.t0, clk.t1 = t0, t0 + 0.1
+    s = clk.summary()
+    assert s["samples"] == 5 and s["sm_mhz"] == 1702.0
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w_max"] == 900.0
+    assert s["sm_max_mhz"] == 1965.0 and s["window_ms"] == 100.0
