@@ -42,8 +42,10 @@ namespace plx {
 
 namespace {
 
-constexpr int kBwdEltWarps = 8;                       // warps 2 .. 9
+constexpr int kBwdEltWarps = 8;                       // rows kernel: warps 2 .. 9
 constexpr int kBwdThreads = (2 + kBwdEltWarps) * 32;  // 320
+constexpr int kKeysEltWarps = 16;                      // keys kernel: warps 2 .. 17
+constexpr int kKeysThreads = (2 + kKeysEltWarps) * 32;  // 576
 constexpr int kBwdStages = 3;                         // ring depth of the streamed operand
 constexpr int kTileM = 128;                           // TMEM lanes: rows (rows kernel) or keys
 constexpr int kTileN = 64;                            // keys (rows kernel) or query rows per step
@@ -478,7 +480,7 @@ struct KeysBars {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kKeysThreads, 1)
     plx_bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                            const __grid_constant__ CUtensorMap rmap,
                            const __grid_constant__ CUtensorMap gmap,
@@ -506,9 +508,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bars->q_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_done, kBwdEltWarps);
+    mbar_init(&bars->s_done, kKeysEltWarps);
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->acc_empty, kBwdEltWarps);
+    mbar_init(&bars->acc_empty, kKeysEltWarps);
     mbar_init(&bars->drain, 1);
     fence_mbarrier_init();
   }
@@ -670,11 +672,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise + epilogue
-    const int half = (warp - 2) >> 2;     // which 32 query columns of each step
+    // sixteen warps: four per TMEM lane quadrant, each thread one key and a
+    // quarter (16 query columns) of every step, which is one k step of the
+    // gradient products
+    const int quarter = (warp - 2) >> 2;  // which 16 query columns of each step
     const int qd = warp & 3;              // TMEM lane quadrant
     const int r = qd * 32 + lane;         // key of the key tile
     const uint32_t lane_addr = tbase + ((uint32_t)(qd * 32) << 16);
-    const uint32_t my = (uint32_t)(half * 32);
+    const uint32_t my = (uint32_t)(quarter * 16);
+    const uint32_t hi_col = packed_col(quarter), lo_col = hi_col + kLoCols;
     const float qs = p.qscale;
     int t = 0, ku = 0;
     for (int k = 0, u; (u = cta_unit(k, p.units)) >= 0; ++k) {
@@ -689,15 +695,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_wait(&bars->q_full[st], (t / kBwdStages) & 1, abort_flag, p.err);
         mbar_wait(&bars->s_full, t & 1, abort_flag, p.err);
         tc_fence_after();
-        uint32_t sv[32], tv[32], gv[32];
-        tmem_ld2x32_sync(lane_addr + C::COL_S + my, lane_addr + C::COL_T + my, sv, tv);
-        tmem_ld32_sync(lane_addr + C::COL_GV + my, gv);
+        uint32_t sv[16], tv[16], gv[16];
+        tmem_ld2x16_sync(lane_addr + C::COL_S + my, lane_addr + C::COL_T + my, sv, tv);
+        tmem_ld16_sync(lane_addr + C::COL_GV + my, gv);
         const float4* stat =
-            reinterpret_cast<const float4*>(sRing + st * STAGE + 3 * C::SMALL) + half * 32;
-        const int i0 = qt * kTileN + half * 32;  // first query column of this half
-        uint32_t pp[32], pds[32], pdt[32];  // [0, 16) high parts, [16, 32) low parts
+            reinterpret_cast<const float4*>(sRing + st * STAGE + 3 * C::SMALL) + quarter * 16;
+        const int i0 = qt * kTileN + quarter * 16;  // first query column of this quarter
+        uint32_t pp[2][8], pds[2][8], pdt[2][8];  // [0]: high parts, [1]: low parts
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < 16; c += 2) {
           float pv2[2], ds2[2], dt2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
@@ -711,31 +717,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             dt2[e] = a * (w.z - g_);
             ds2[e] = p.scale * a * fmaf(cc, g_, fmaf(tt, w.z, -w.w));
           }
-          split_bf16(pv2[0], pv2[1], pp[c >> 1], pp[16 + (c >> 1)]);
-          split_bf16(ds2[0], ds2[1], pds[c >> 1], pds[16 + (c >> 1)]);
-          split_bf16(dt2[0], dt2[1], pdt[c >> 1], pdt[16 + (c >> 1)]);
+          split_bf16(pv2[0], pv2[1], pp[0][c >> 1], pp[1][c >> 1]);
+          split_bf16(ds2[0], ds2[1], pds[0][c >> 1], pds[1][c >> 1]);
+          split_bf16(dt2[0], dt2[1], pdt[0][c >> 1], pdt[1][c >> 1]);
         }
-        tmem_st32(lane_addr + C::COL_S + my, pp);
-        tmem_st32(lane_addr + C::COL_T + my, pds);
-        tmem_st32(lane_addr + C::COL_GV + my, pdt);
+        tmem_st8(lane_addr + C::COL_S + hi_col, pp[0]);
+        tmem_st8(lane_addr + C::COL_S + lo_col, pp[1]);
+        tmem_st8(lane_addr + C::COL_T + hi_col, pds[0]);
+        tmem_st8(lane_addr + C::COL_T + lo_col, pds[1]);
+        tmem_st8(lane_addr + C::COL_GV + hi_col, pdt[0]);
+        tmem_st8(lane_addr + C::COL_GV + lo_col, pdt[1]);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_done);
       }
-      // epilogue: dV, dK of this key (this half's columns), fp32
+      // epilogue: dV, dK of this key (this quarter's columns), fp32
       mbar_wait(&bars->acc_full, ku & 1, abort_flag, p.err);
       tc_fence_after();
       const size_t ro = (((size_t)b * p.L + j) * p.Hkv + hk) * D;
 #pragma unroll 1
-      for (int cc = half * (D / 2); cc < (half + 1) * (D / 2); cc += 32) {
-        uint32_t a0[32], a1[32];
-        tmem_ld2x32_sync(lane_addr + C::COL_A0 + cc, lane_addr + C::COL_A1 + cc, a0, a1);
+      for (int cc = quarter * (D / 4); cc < (quarter + 1) * (D / 4); cc += 16) {
+        uint32_t a0[16], a1[16];
+        tmem_ld2x16_sync(lane_addr + C::COL_A0 + cc, lane_addr + C::COL_A1 + cc, a0, a1);
         if (j < p.L) {
           float4* d0 = reinterpret_cast<float4*>(p.dv + ro + cc);
           float4* d1 = reinterpret_cast<float4*>(p.dk + ro + cc);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
+          for (int q = 0; q < 4; ++q) {
             d0[q] = make_float4(__uint_as_float(a0[4 * q]), __uint_as_float(a0[4 * q + 1]),
                                 __uint_as_float(a0[4 * q + 2]), __uint_as_float(a0[4 * q + 3]));
             d1[q] = make_float4(__uint_as_float(a1[4 * q]), __uint_as_float(a1[4 * q + 1]),
@@ -837,7 +846,7 @@ cudaError_t launch_bwd_tc_d(const BwdTcArgs& a, cudaStream_t stream) {
   e = cudaFuncSetAttribute(keys, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const unsigned keys_grid = (unsigned)(keys_units < a.num_sms ? keys_units : a.num_sms);
-  keys<<<keys_grid, kBwdThreads, smem, stream>>>(qm, rm, gm, km, vm, p);
+  keys<<<keys_grid, kKeysThreads, smem, stream>>>(qm, rm, gm, km, vm, p);
   return cudaGetLastError();
 }
 
