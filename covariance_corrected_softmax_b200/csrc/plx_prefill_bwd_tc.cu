@@ -15,10 +15,10 @@
 // Two kernels, no atomics:
 //  rows  one CTA per (batch, query head, 128-row query tile), two passes over
 //        the row's 64-key tiles.  Pass 1: S = Q K^T, T = R K^T, GV = G V^T;
-//        thread (row, half) runs an online softmax over its half of every key
-//        tile, with sum a, sum a t, sum a gv and sum a t gv; the two halves
-//        merge at the end into the row statistics (lse, tbar, go, D), which go
-//        to the workspace.  Pass 2: S, T, GV again; ds and dt, as high and low
+//        thread (row, quarter) runs an online softmax over its quarter of
+//        every key tile, with sum a, sum a t, sum a gv and sum a t gv; the four
+//        quarters merge at the end into the row statistics (lse, tbar, go, D),
+//        which go to the workspace.  Pass 2: S, T, GV again; ds and dt, as high and low
 //        bf16 parts, are written over S and T in TMEM, and dQ += (scale ds) K,
 //        dR += dt K accumulate in TMEM.
 //  keys  one CTA per (batch, kv head, 128-key tile), over the query heads of
@@ -31,8 +31,9 @@
 // forward pass): ds = a (X - D) cancels where one key dominates a row, and
 // would amplify any rounding of the normaliser.
 // Per CTA: warp 0 issues the TMA loads, warp 1 (one thread) the MMAs and owns
-// the TMEM columns, warps 2-9 do the elementwise work (thread = TMEM lane and
-// half of a tile's columns) and the epilogue.  The products of a step are
+// the TMEM columns, warps 2-17 do the elementwise work (thread = TMEM lane and
+// a quarter of a tile's columns, four warps per lane quadrant) and the
+// epilogue.  The products of a step are
 // issued once the elementwise warps have stored their operands, and the next
 // step's S/T/GV after them, so the tensor core never overwrites a column that
 // is still to be read.
@@ -42,10 +43,10 @@ namespace plx {
 
 namespace {
 
-constexpr int kBwdEltWarps = 8;                       // rows kernel: warps 2 .. 9
-constexpr int kBwdThreads = (2 + kBwdEltWarps) * 32;  // 320
-constexpr int kKeysEltWarps = 16;                      // keys kernel: warps 2 .. 17
-constexpr int kKeysThreads = (2 + kKeysEltWarps) * 32;  // 576
+// Elementwise warps 2 .. 17: four per TMEM lane quadrant, each thread one
+// TMEM lane and a quarter (16 columns) of every tile or step.
+constexpr int kBwdEltWarps = 16;
+constexpr int kBwdThreads = (2 + kBwdEltWarps) * 32;  // 576
 constexpr int kBwdStages = 3;                         // ring depth of the streamed operand
 constexpr int kTileM = 128;                           // TMEM lanes: rows (rows kernel) or keys
 constexpr int kTileN = 64;                            // keys (rows kernel) or query rows per step
@@ -81,9 +82,11 @@ struct BwdCfg {
 };
 
 // Column of the bf16 pairs of columns [16 kk, 16 kk + 16) of a 64-column S/T/GV
-// block once the elementwise warps have written their operand over it: half h
-// packs the high bf16 parts of its 32 columns into the first 16 of its own 32
-// and the low parts (value - high, rounded) into the next 16 (+kLoCols).  The
+// block once the elementwise warps have written their operand over it: the
+// thread of quarter kk writes the high bf16 parts of its 16 columns at
+// packed_col(kk) and the low parts (value - high, rounded) 16 columns further
+// (+kLoCols), so each half of the block holds the high parts of its two
+// quarters in its first 16 columns and their low parts in the next 16.  The
 // gradient products run once on each part, so the operands keep about 16
 // significant bits: the fp32 gradients' own error, not bf16's.
 __device__ __forceinline__ uint32_t packed_col(int kk) {
@@ -165,8 +168,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* sR = smem + C::BIG;
   uint8_t* sG = smem + 2 * C::BIG;
   uint8_t* sKV = smem + 3 * C::BIG;  // stage st: K at st * 2 SMALL, V after it
-  float* xch = reinterpret_cast<float*>(sKV + kBwdStages * 2 * C::SMALL);  // [5][2][128]
-  RowsBars* bars = reinterpret_cast<RowsBars*>(xch + 5 * 2 * kTileM);
+  float* xch = reinterpret_cast<float*>(sKV + kBwdStages * 2 * C::SMALL);  // [5][4][128]
+  RowsBars* bars = reinterpret_cast<RowsBars*>(xch + 5 * 4 * kTileM);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -329,11 +332,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise + epilogue
-    const int half = (warp - 2) >> 2;     // which 32 columns of each tile
+    const int quarter = (warp - 2) >> 2;  // which 16 columns of each tile
     const int qd = warp & 3;              // TMEM lane quadrant
     const int r = qd * 32 + lane;         // row of the query tile
     const uint32_t lane_addr = tbase + ((uint32_t)(qd * 32) << 16);
-    const uint32_t my = (uint32_t)(half * 32);
+    const uint32_t my = (uint32_t)(quarter * 16);
+    const uint32_t hi_col = packed_col(quarter), lo_col = hi_col + kLoCols;
     const float qs = p.qscale;
     int t = 0, ku = 0;
     for (int k = 0, u; (u = cta_unit(k, p.units)) >= 0; ++k) {
@@ -341,22 +345,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       unit_of(u, b, h, mt, n);
       const int i = mt * kTileM + r;
       const int lim = p.causal ? i : p.L - 1;  // last key the row sees
-      // pass 1: online softmax over this half of every key tile (log2 units)
+      // pass 1: online softmax over this quarter of every key tile (log2 units)
       float m = -INFINITY, l = 0.f, st_ = 0.f, sg = 0.f, stg = 0.f;
       for (int j = 0; j < n; ++j, ++t) {
         mbar_wait(&bars->s_full, t & 1, abort_flag, p.err);
         tc_fence_after();
-        uint32_t sv[32], tv[32], gv[32];
-        tmem_ld2x32_sync(lane_addr + C::COL_S + my, lane_addr + C::COL_T + my, sv, tv);
-        tmem_ld32_sync(lane_addr + C::COL_GV + my, gv);
+        uint32_t sv[16], tv[16], gv[16];
+        tmem_ld2x16_sync(lane_addr + C::COL_S + my, lane_addr + C::COL_T + my, sv, tv);
+        tmem_ld16_sync(lane_addr + C::COL_GV + my, gv);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_done);
-        const int nvis = max(0, min(32, lim - (j * kTileN + half * 32) + 1));
-        float x[32];
+        const int nvis = max(0, min(16, lim - (j * kTileN + quarter * 16) + 1));
+        float x[16];
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < 16; ++c) {
           x[c] = __uint_as_float(sv[c]) * qs;
           if (c < nvis) mx = fmaxf(mx, x[c]);
         }
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           m = mx;
         }
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < 16; ++c) {
           const float e = c < nvis ? exp2f(x[c] - m) : 0.f;
           const float tt = __uint_as_float(tv[c]), g_ = __uint_as_float(gv[c]);
           l += e;
@@ -378,41 +382,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           stg = fmaf(e * tt, g_, stg);
         }
       }
-      // merge the two halves of the row
+      // merge the four quarters of the row
       {
-        float* w = xch + half * kTileM + r;
+        float* w = xch + quarter * kTileM + r;
         w[0] = m;
-        w[2 * kTileM] = l;
-        w[4 * kTileM] = st_;
-        w[6 * kTileM] = sg;
-        w[8 * kTileM] = stg;
+        w[4 * kTileM] = l;
+        w[8 * kTileM] = st_;
+        w[12 * kTileM] = sg;
+        w[16 * kTileM] = stg;
       }
-      named_bar_sync(1 + qd, 64);
-      const float* o = xch + (half ^ 1) * kTileM + r;
-      const float m2 = o[0];
-      const float M = fmaxf(m, m2);
-      const float fa = m == -INFINITY ? 0.f : exp2f(m - M);
-      const float fb = m2 == -INFINITY ? 0.f : exp2f(m2 - M);
-      const float L_ = l * fa + o[2 * kTileM] * fb;
+      named_bar_sync(1 + qd, 128);
+      float mq[4], M = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        mq[q] = xch[q * kTileM + r];
+        M = fmaxf(M, mq[q]);
+      }
+      float L_ = 0.f, st_all = 0.f, sg_all = 0.f, stg_all = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float f = mq[q] == -INFINITY ? 0.f : exp2f(mq[q] - M);
+        const float* o = xch + q * kTileM + r;
+        L_ = fmaf(o[4 * kTileM], f, L_);
+        st_all = fmaf(o[8 * kTileM], f, st_all);
+        sg_all = fmaf(o[12 * kTileM], f, sg_all);
+        stg_all = fmaf(o[16 * kTileM], f, stg_all);
+      }
       const float inv = 1.f / L_;
       const float lse2 = M + log2f(L_);
-      const float tbar = (st_ * fa + o[4 * kTileM] * fb) * inv;
-      const float go = (sg * fa + o[6 * kTileM] * fb) * inv;
-      const float wsum = (stg * fa + o[8 * kTileM] * fb) * inv;
+      const float tbar = st_all * inv;
+      const float go = sg_all * inv;
+      const float wsum = stg_all * inv;
       const float Dr = (1.f + 2.f * tbar) * go - wsum;
-      if (half == 0 && i < p.L)
+      if (quarter == 0 && i < p.L)
         p.stats[((size_t)b * p.Hq + h) * p.L + i] = make_float4(lse2, tbar, go, Dr);
       // pass 2: scale ds and dt, rounded to bf16, over S and T
       for (int j = 0; j < n; ++j, ++t) {
         mbar_wait(&bars->s_full, t & 1, abort_flag, p.err);
         tc_fence_after();
-        uint32_t sv[32], tv[32], gv[32];
-        tmem_ld2x32_sync(lane_addr + C::COL_S + my, lane_addr + C::COL_T + my, sv, tv);
-        tmem_ld32_sync(lane_addr + C::COL_GV + my, gv);
-        const int nvis = max(0, min(32, lim - (j * kTileN + half * 32) + 1));
-        uint32_t pds[32], pdt[32];  // [0, 16) high parts, [16, 32) low parts
+        uint32_t sv[16], tv[16], gv[16];
+        tmem_ld2x16_sync(lane_addr + C::COL_S + my, lane_addr + C::COL_T + my, sv, tv);
+        tmem_ld16_sync(lane_addr + C::COL_GV + my, gv);
+        const int nvis = max(0, min(16, lim - (j * kTileN + quarter * 16) + 1));
+        uint32_t pds[2][8], pdt[2][8];  // [0]: high parts, [1]: low parts
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < 16; c += 2) {
           float ds2[2], dt2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
@@ -423,29 +437,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             dt2[e] = a * (go - g_);
             ds2[e] = p.scale * a * fmaf(cc, g_, fmaf(tt, go, -Dr));
           }
-          split_bf16(ds2[0], ds2[1], pds[c >> 1], pds[16 + (c >> 1)]);
-          split_bf16(dt2[0], dt2[1], pdt[c >> 1], pdt[16 + (c >> 1)]);
+          split_bf16(ds2[0], ds2[1], pds[0][c >> 1], pds[1][c >> 1]);
+          split_bf16(dt2[0], dt2[1], pdt[0][c >> 1], pdt[1][c >> 1]);
         }
-        tmem_st32(lane_addr + C::COL_S + my, pds);
-        tmem_st32(lane_addr + C::COL_T + my, pdt);
+        tmem_st8(lane_addr + C::COL_S + hi_col, pds[0]);
+        tmem_st8(lane_addr + C::COL_S + lo_col, pds[1]);
+        tmem_st8(lane_addr + C::COL_T + hi_col, pdt[0]);
+        tmem_st8(lane_addr + C::COL_T + lo_col, pdt[1]);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_done);
       }
-      // epilogue: dQ, dR of this row (this half's columns), fp32
+      // epilogue: dQ, dR of this row (this quarter's columns), fp32
       mbar_wait(&bars->acc_full, ku & 1, abort_flag, p.err);
       tc_fence_after();
       const size_t ro = (((size_t)b * p.L + i) * p.Hq + h) * D;
 #pragma unroll 1
-      for (int cc = half * (D / 2); cc < (half + 1) * (D / 2); cc += 32) {
-        uint32_t a0[32], a1[32];
-        tmem_ld2x32_sync(lane_addr + C::COL_A0 + cc, lane_addr + C::COL_A1 + cc, a0, a1);
+      for (int cc = quarter * (D / 4); cc < (quarter + 1) * (D / 4); cc += 16) {
+        uint32_t a0[16], a1[16];
+        tmem_ld2x16_sync(lane_addr + C::COL_A0 + cc, lane_addr + C::COL_A1 + cc, a0, a1);
         if (i < p.L) {
           float4* d0 = reinterpret_cast<float4*>(p.dq + ro + cc);
           float4* d1 = reinterpret_cast<float4*>(p.drho + ro + cc);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
+          for (int q = 0; q < 4; ++q) {
             d0[q] = make_float4(__uint_as_float(a0[4 * q]), __uint_as_float(a0[4 * q + 1]),
                                 __uint_as_float(a0[4 * q + 2]), __uint_as_float(a0[4 * q + 3]));
             d1[q] = make_float4(__uint_as_float(a1[4 * q]), __uint_as_float(a1[4 * q + 1]),
@@ -480,7 +496,7 @@ struct KeysBars {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kKeysThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     plx_bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                            const __grid_constant__ CUtensorMap rmap,
                            const __grid_constant__ CUtensorMap gmap,
@@ -508,9 +524,9 @@ __global__ void __launch_bounds__(kKeysThreads, 1)
       mbar_init(&bars->q_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_done, kKeysEltWarps);
+    mbar_init(&bars->s_done, kBwdEltWarps);
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->acc_empty, kKeysEltWarps);
+    mbar_init(&bars->acc_empty, kBwdEltWarps);
     mbar_init(&bars->drain, 1);
     fence_mbarrier_init();
   }
@@ -709,7 +725,10 @@ __global__ void __launch_bounds__(kKeysThreads, 1)
           for (int e = 0; e < 2; ++e) {
             const int i = i0 + c + e;
             const bool vis = i < p.L && j < p.L && (!p.causal || i >= j);
-            const float4 w = stat[c + e];  // lse (log2), tbar, go, D of query i
+            // lse (log2), tbar, go, D of query i; a query past L has no
+            // statistics (its ring slot holds whatever was there), and a zero
+            // weight must not meet a non-finite value
+            const float4 w = vis ? stat[c + e] : make_float4(0.f, 0.f, 0.f, 0.f);
             const float a = vis ? exp2f(fmaf(__uint_as_float(sv[c + e]), qs, -w.x)) : 0.f;
             const float tt = __uint_as_float(tv[c + e]), g_ = __uint_as_float(gv[c + e]);
             const float cc = 1.f + w.y - tt;
@@ -784,7 +803,7 @@ cudaError_t encode_bwd_map(CUtensorMap* map, const void* base, int B, int L, int
 template <int D>
 constexpr int rows_smem_bytes() {
   using C = BwdCfg<D>;
-  return 1024 + 3 * C::BIG + kBwdStages * 2 * C::SMALL + 5 * 2 * kTileM * 4 +
+  return 1024 + 3 * C::BIG + kBwdStages * 2 * C::SMALL + 5 * 4 * kTileM * 4 +
          (int)sizeof(RowsBars) + 16;
 }
 template <int D>
@@ -846,7 +865,7 @@ cudaError_t launch_bwd_tc_d(const BwdTcArgs& a, cudaStream_t stream) {
   e = cudaFuncSetAttribute(keys, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const unsigned keys_grid = (unsigned)(keys_units < a.num_sms ? keys_units : a.num_sms);
-  keys<<<keys_grid, kKeysThreads, smem, stream>>>(qm, rm, gm, km, vm, p);
+  keys<<<keys_grid, kBwdThreads, smem, stream>>>(qm, rm, gm, km, vm, p);
   return cudaGetLastError();
 }
 
