@@ -39,13 +39,18 @@ def _check_projection(got, x, w, bf16):
 # On 148 SMs the bf16 shapes reach each schedule: one tile (1x64x64,
 # 128x136x64), clusters of CTAs splitting K (5x256x72, 300x2048x2048,
 # 1000x384x520 with an uneven split, 32x2048x2048 the decode batch),
-# persistent single tiles (2000x1024x256) and pairs of tiles with an odd last
-# tile and ragged M, N, K (4100x1032x200).
+# persistent single tiles (2000x1024x256), persistent pairs of tiles with an
+# odd last tile and ragged M, N, K (2100x1096x136), SM pairs with ragged M, N,
+# K and more 256 x 256 tiles than pairs (4100x1032x200); the smallest N and K
+# the tensor cores take (3x8x16, 129x264x8: one partial tile and one partial
+# k block).
 @pytest.mark.parametrize("M,N,K", [(1, 64, 64), (5, 256, 72), (128, 136, 64), (300, 2048, 2048),
                                    (1000, 384, 520), (32, 2048, 2048), (2000, 1024, 256),
-                                   (4100, 1032, 200)],
+                                   (4100, 1032, 200), (2100, 1096, 136), (3, 8, 16),
+                                   (129, 264, 8)],
                          ids=["1x64x64", "5x256x72", "128x136x64", "300x2048x2048", "1000x384x520",
-                              "32x2048x2048", "2000x1024x256", "4100x1032x200"])
+                              "32x2048x2048", "2000x1024x256", "4100x1032x200", "2100x1096x136",
+                              "3x8x16", "129x264x8"])
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
 def test_projection_matches_oracle(M, N, K, dt):
     x, w = W.make_probe_inputs((M,), K, N, seed=M + N + K, device=DEV, dtype=dt)
